@@ -1,0 +1,115 @@
+"""ctypes binding of libpuro_fp8.so: the C ABI of include/puro_fp8.h, same names.
+
+Argument marshalling only.  Every pointer is an integer device address and
+every stream an integer cudaStream_t.  There is no fallback: if the library is
+missing or the device is not a B200 the calls fail loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpuro_fp8.so")
+
+PURO_OK = 0
+PURO_ERR_NULL = -1
+PURO_ERR_ALIGN = -2
+PURO_ERR_SHAPE = -3
+PURO_ERR_LAYOUT = -4
+PURO_ERR_CUDA = -5
+PURO_ERR_UNSUPPORTED_DEVICE = -6
+PURO_ERR_DEVICE_TIMEOUT = -7
+
+PURO_ROWWISE = 1
+PURO_COLWISE = 2
+PURO_BOTH = 3
+
+EXPORTS = (
+    "puro_fp8_quant_act",
+    "puro_fp8_quant_weight",
+    "puro_fp8_gemm_fprop",
+    "puro_fp8_gemm_dgrad",
+    "puro_fp8_gemm_wgrad",
+    "puro_fp8_device_status",
+    "puro_fp8_status_string",
+    "puro_fp8_test_bounded_wait",
+)
+
+_lib = None
+
+
+class PuroError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = status
+        super().__init__("%s%s" % (where + ": " if where else "", status_string(status)))
+
+
+def load() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            "libpuro_fp8.so is missing (%s); build it with "
+            "`python -c 'import __graft_entry__ as g; g.build()'`" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.puro_fp8_quant_act.argtypes = [P, I, I, I, INT, P, I, P, I, P, I, P, I, P]
+    lib.puro_fp8_quant_weight.argtypes = [P, I, I, I, P, I, P, P, I, P]
+    lib.puro_fp8_gemm_fprop.argtypes = [P, I, P, I, P, I, P, P, I, I, I, I, P]
+    lib.puro_fp8_gemm_dgrad.argtypes = [P, I, P, I, P, I, P, P, I, I, I, I, P]
+    lib.puro_fp8_gemm_wgrad.argtypes = [P, I, P, I, P, I, P, I, P, I, I, I, I, P]
+    lib.puro_fp8_device_status.argtypes = [P]
+    lib.puro_fp8_status_string.argtypes = [INT]
+    lib.puro_fp8_status_string.restype = ctypes.c_char_p
+    lib.puro_fp8_test_bounded_wait.argtypes = [I, P]
+    for name in EXPORTS:
+        if name != "puro_fp8_status_string":
+            getattr(lib, name).restype = INT
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().puro_fp8_status_string(int(status)).decode()
+
+
+def puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, ld_s, qt, ld_qt, st, ld_st,
+                       stream) -> int:
+    return load().puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, ld_s, qt, ld_qt,
+                                     st, ld_st, stream)
+
+
+def puro_fp8_quant_weight(w, n, k, ld_w, q, ld_q, s, qt, ld_qt, stream) -> int:
+    return load().puro_fp8_quant_weight(w, n, k, ld_w, q, ld_q, s, qt, ld_qt, stream)
+
+
+def puro_fp8_gemm_fprop(qx, ld_qx, sx, ld_sx, qw, ld_qw, sw, y, ld_y, m, n, k, stream) -> int:
+    return load().puro_fp8_gemm_fprop(qx, ld_qx, sx, ld_sx, qw, ld_qw, sw, y, ld_y, m, n, k,
+                                      stream)
+
+
+def puro_fp8_gemm_dgrad(qdy, ld_qdy, sdy, ld_sdy, qwt, ld_qwt, sw, dx, ld_dx, m, n, k,
+                        stream) -> int:
+    return load().puro_fp8_gemm_dgrad(qdy, ld_qdy, sdy, ld_sdy, qwt, ld_qwt, sw, dx, ld_dx, m, n,
+                                      k, stream)
+
+
+def puro_fp8_gemm_wgrad(qdyt, ld_qdyt, sdyt, ld_sdyt, qxt, ld_qxt, sxt, ld_sxt, dw, ld_dw, m, n,
+                        k, stream) -> int:
+    return load().puro_fp8_gemm_wgrad(qdyt, ld_qdyt, sdyt, ld_sdyt, qxt, ld_qxt, sxt, ld_sxt, dw,
+                                      ld_dw, m, n, k, stream)
+
+
+def puro_fp8_device_status(stream) -> int:
+    return load().puro_fp8_device_status(stream)
+
+
+def puro_fp8_status_string(status) -> str:
+    return status_string(status)
+
+
+def puro_fp8_test_bounded_wait(limit_ns, stream) -> int:
+    return load().puro_fp8_test_bounded_wait(limit_ns, stream)

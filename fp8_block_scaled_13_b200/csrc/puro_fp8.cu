@@ -1,0 +1,373 @@
+// C ABI of the block-scaled FP8 linear layer (declared in include/puro_fp8.h).
+//
+// Host side: argument validation (before any CUDA call), device check
+// (sm_100 only), TMA tensor-map encoding through the driver entry point
+// (no link against libcuda), and kernel launches on the caller's stream.
+// All kernels live in this one translation unit so that they share the
+// device error word.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/puro_fp8.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool checked = false;
+  bool supported = false;
+  int sms = 0;
+  bool attrs_set = false;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device: must be compute capability 10.0 (B200, sm_100a).
+int current_device(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PURO_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return PURO_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.sms = sms;
+    d.checked = true;
+  }
+  if (!d.supported) return PURO_ERR_UNSUPPORTED_DEVICE;
+  *out = &d;
+  return PURO_OK;
+}
+
+int get_encoder() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_encode) return PURO_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return PURO_ERR_CUDA;
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return PURO_OK;
+}
+
+// 2-D byte tensor [outer, inner] with row stride `ld` bytes; box {box_inner,
+// box_outer}; optional 128-byte swizzle; out-of-range reads return zero.
+int make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+                uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PURO_OK : PURO_ERR_CUDA;
+}
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? PURO_OK : PURO_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ quant
+
+template <bool ROW, bool COL, bool BLOCK>
+int launch_quant(const puro::QuantParams& p, int sms, cudaStream_t stream) {
+  const int64_t grid = p.tiles < (int64_t)sms * 8 ? p.tiles : (int64_t)sms * 8;
+  puro::quant_tile_kernel<ROW, COL, BLOCK><<<(unsigned)grid, 256, 0, stream>>>(p);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ gemm
+
+struct GemmArgs {
+  const void* a;    int64_t lda;     // E4M3 [rows_a, K]
+  const void* sfa;  int64_t ld_sfa;  // group-major [KB][ld_sfa]
+  const void* b;    int64_t ldb;     // E4M3 [rows_b, K]
+  const void* sfb;  int64_t ld_sfb;  // per-row: group-major [KB][ld_sfb]
+  bool b_per_row;
+  const uint8_t* bsf; int64_t bsf_row, bsf_col;  // per-block scales of B
+  void* d; int64_t ldd;
+  int64_t rows_a, rows_b, k;
+};
+
+template <int BN, bool PER_ROW>
+int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
+  using C = puro::GemmCfg<BN>;
+  CUtensorMap ma, mb, msa, msb;
+  const uint64_t kb = (uint64_t)((g.k + 127) / 128);
+  int st;
+  if ((st = make_map_u8(&ma, g.a, g.k, g.rows_a, g.lda, 128, 128, true)) != PURO_OK) return st;
+  if ((st = make_map_u8(&mb, g.b, g.k, g.rows_b, g.ldb, 128, BN, true)) != PURO_OK) return st;
+  if ((st = make_map_u8(&msa, g.sfa, g.rows_a, kb, g.ld_sfa, 128, 1, false)) != PURO_OK) return st;
+  if (PER_ROW) {
+    if ((st = make_map_u8(&msb, g.sfb, g.rows_b, kb, g.ld_sfb, BN, 1, false)) != PURO_OK) return st;
+  } else {
+    msb = msa;  // unused by the kernel
+  }
+  auto kern = puro::gemm_block_scaled_kernel<BN, PER_ROW>;
+  static bool attr_done[kMaxDevices] = {};
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  if (!attr_done[dev_id]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+      return PURO_ERR_CUDA;
+    attr_done[dev_id] = true;
+  }
+  puro::GemmParams p;
+  p.rows_a = (int32_t)g.rows_a;
+  p.rows_b = (int32_t)g.rows_b;
+  p.kblocks = (int32_t)kb;
+  p.tiles_m = (int32_t)((g.rows_a + 127) / 128);
+  p.tiles_n = (int32_t)((g.rows_b + BN - 1) / BN);
+  p.bsf = g.bsf;
+  p.bsf_row = (int32_t)g.bsf_row;
+  p.bsf_col = (int32_t)g.bsf_col;
+  p.d = reinterpret_cast<__nv_bfloat16*>(g.d);
+  p.ldd = g.ldd;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < dev->sms ? tiles : dev->sms;
+  kern<<<grid, 192, C::kSmemBytes, stream>>>(ma, mb, msa, msb, p);
+  return launch_status();
+}
+
+int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != PURO_OK) return st;
+  if ((st = get_encoder()) != PURO_OK) return st;
+  if (g.rows_a == 0 || g.rows_b == 0) return PURO_OK;
+  if (g.k == 0) {
+    // empty reduction: the product is exactly zero
+    if (cudaMemset2DAsync(g.d, (size_t)g.ldd * 2, 0, (size_t)g.rows_b * 2, (size_t)g.rows_a,
+                          stream) != cudaSuccess)
+      return PURO_ERR_CUDA;
+    return PURO_OK;
+  }
+  if (g.b_per_row) return launch_gemm_cfg<256, true>(g, dev, stream);
+  return launch_gemm_cfg<256, false>(g, dev, stream);
+}
+
+// Shape/alignment checks shared by the three GEMMs.
+int check_mat(const void* p, int64_t ld, int64_t min_ld, int64_t elem_bytes) {
+  if (!p) return PURO_ERR_NULL;
+  if (!aligned16(p)) return PURO_ERR_ALIGN;
+  if (ld < min_ld) return PURO_ERR_SHAPE;
+  if ((ld * elem_bytes) % 16) return PURO_ERR_ALIGN;
+  return PURO_OK;
+}
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+
+}  // namespace
+
+extern "C" {
+
+const char* puro_fp8_status_string(int status) {
+  switch (status) {
+    case PURO_OK: return "PURO_OK";
+    case PURO_ERR_NULL: return "PURO_ERR_NULL: a required pointer is NULL";
+    case PURO_ERR_ALIGN: return "PURO_ERR_ALIGN: pointer or leading dimension not 16-byte aligned";
+    case PURO_ERR_SHAPE: return "PURO_ERR_SHAPE: size or leading dimension out of range";
+    case PURO_ERR_LAYOUT: return "PURO_ERR_LAYOUT: unknown layout flag";
+    case PURO_ERR_CUDA: return "PURO_ERR_CUDA: a CUDA call failed";
+    case PURO_ERR_UNSUPPORTED_DEVICE: return "PURO_ERR_UNSUPPORTED_DEVICE: needs sm_100 (B200)";
+    case PURO_ERR_DEVICE_TIMEOUT: return "PURO_ERR_DEVICE_TIMEOUT: a bounded device wait expired";
+    default: return "unknown puro_status";
+  }
+}
+
+int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int layout,
+                       void* q, int64_t ld_q, void* s, int64_t ld_s, void* qt, int64_t ld_qt,
+                       void* st, int64_t ld_st, void* stream) {
+  if (layout != PURO_ROWWISE && layout != PURO_COLWISE && layout != PURO_BOTH)
+    return PURO_ERR_LAYOUT;
+  if (rows < 0 || cols < 0 || rows >= kMaxDim || cols >= kMaxDim) return PURO_ERR_SHAPE;
+  if (cols % 128) return PURO_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return PURO_OK;
+  int r;
+  if ((r = check_mat(x, ld_x, cols, 2)) != PURO_OK) return r;
+  const bool row = layout & PURO_ROWWISE, col = layout & PURO_COLWISE;
+  if (row) {
+    if ((r = check_mat(q, ld_q, cols, 1)) != PURO_OK) return r;
+    if ((r = check_mat(s, ld_s, rows, 1)) != PURO_OK) return r;
+  }
+  if (col) {
+    if ((r = check_mat(qt, ld_qt, (rows + 15) / 16 * 16, 1)) != PURO_OK) return r;
+    if ((r = check_mat(st, ld_st, cols, 1)) != PURO_OK) return r;
+  }
+  DeviceInfo* dev = nullptr;
+  if ((r = current_device(&dev)) != PURO_OK) return r;
+  puro::QuantParams p{};
+  p.x = static_cast<const uint16_t*>(x);
+  p.rows = rows;
+  p.cols = cols;
+  p.ld_x = ld_x;
+  p.q = static_cast<uint8_t*>(q);
+  p.ld_q = ld_q;
+  p.s = static_cast<uint8_t*>(s);
+  p.ld_s = ld_s;
+  p.qt = static_cast<uint8_t*>(qt);
+  p.ld_qt = ld_qt;
+  p.st = static_cast<uint8_t*>(st);
+  p.ld_st = ld_st;
+  p.tiles_c = cols / 128;
+  p.tiles = p.tiles_c * ((rows + 127) / 128);
+  cudaStream_t sm = static_cast<cudaStream_t>(stream);
+  if (row && col) return launch_quant<true, true, false>(p, dev->sms, sm);
+  if (row) return launch_quant<true, false, false>(p, dev->sms, sm);
+  return launch_quant<false, true, false>(p, dev->sms, sm);
+}
+
+int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, void* q, int64_t ld_q,
+                          void* s, void* qt, int64_t ld_qt, void* stream) {
+  if (n < 0 || k < 0 || n >= kMaxDim || k >= kMaxDim || n % 128 || k % 128) return PURO_ERR_SHAPE;
+  if (n == 0 || k == 0) return PURO_OK;
+  int r;
+  if ((r = check_mat(w, ld_w, k, 2)) != PURO_OK) return r;
+  if ((r = check_mat(q, ld_q, k, 1)) != PURO_OK) return r;
+  if (!s) return PURO_ERR_NULL;
+  if (qt && (r = check_mat(qt, ld_qt, n, 1)) != PURO_OK) return r;
+  DeviceInfo* dev = nullptr;
+  if ((r = current_device(&dev)) != PURO_OK) return r;
+  puro::QuantParams p{};
+  p.x = static_cast<const uint16_t*>(w);
+  p.rows = n;
+  p.cols = k;
+  p.ld_x = ld_w;
+  p.q = static_cast<uint8_t*>(q);
+  p.ld_q = ld_q;
+  p.qt = static_cast<uint8_t*>(qt);
+  p.ld_qt = ld_qt;
+  p.sw = static_cast<uint8_t*>(s);
+  p.tiles_c = k / 128;
+  p.tiles = p.tiles_c * (n / 128);
+  cudaStream_t sm = static_cast<cudaStream_t>(stream);
+  if (qt) return launch_quant<true, true, true>(p, dev->sms, sm);
+  return launch_quant<true, false, true>(p, dev->sms, sm);
+}
+
+int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx, int64_t ld_sx,
+                        const void* qw, int64_t ld_qw, const void* sw, void* y, int64_t ld_y,
+                        int64_t m, int64_t n, int64_t k, void* stream) {
+  if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
+  if (n % 128 || k % 128) return PURO_ERR_SHAPE;
+  if (k / 128 > puro::GemmCfg<256>::kPanel / puro::GemmCfg<256>::kNB) return PURO_ERR_SHAPE;
+  if (m == 0 || n == 0) return PURO_OK;
+  int r;
+  if ((r = check_mat(y, ld_y, n, 2)) != PURO_OK) return r;
+  if (k > 0) {
+    if ((r = check_mat(qx, ld_qx, k, 1)) != PURO_OK) return r;
+    if ((r = check_mat(sx, ld_sx, m, 1)) != PURO_OK) return r;
+    if ((r = check_mat(qw, ld_qw, k, 1)) != PURO_OK) return r;
+    if (!sw) return PURO_ERR_NULL;
+  }
+  GemmArgs g{qx, ld_qx, sx, ld_sx, qw, ld_qw, nullptr, 0, false,
+             static_cast<const uint8_t*>(sw), k / 128, 1, y, ld_y, m, n, k};
+  return launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+int puro_fp8_gemm_dgrad(const void* qdy, int64_t ld_qdy, const void* sdy, int64_t ld_sdy,
+                        const void* qwt, int64_t ld_qwt, const void* sw, void* dx, int64_t ld_dx,
+                        int64_t m, int64_t n, int64_t k, void* stream) {
+  if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
+  if (n % 128 || k % 128) return PURO_ERR_SHAPE;
+  if (n / 128 > puro::GemmCfg<256>::kPanel / puro::GemmCfg<256>::kNB) return PURO_ERR_SHAPE;
+  if (m == 0 || k == 0) return PURO_OK;
+  int r;
+  if ((r = check_mat(dx, ld_dx, k, 2)) != PURO_OK) return r;
+  if (n > 0) {
+    if ((r = check_mat(qdy, ld_qdy, n, 1)) != PURO_OK) return r;
+    if ((r = check_mat(sdy, ld_sdy, m, 1)) != PURO_OK) return r;
+    if ((r = check_mat(qwt, ld_qwt, n, 1)) != PURO_OK) return r;
+    if (!sw) return PURO_ERR_NULL;
+  }
+  // B = W^T [k, n]; its (row j = k-index, group kb = n-block) scale is
+  // sw[kb * (k/128) + j/128].
+  GemmArgs g{qdy, ld_qdy, sdy, ld_sdy, qwt, ld_qwt, nullptr, 0, false,
+             static_cast<const uint8_t*>(sw), 1, k / 128, dx, ld_dx, m, k, n};
+  return launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* sdyt, int64_t ld_sdyt,
+                        const void* qxt, int64_t ld_qxt, const void* sxt, int64_t ld_sxt, void* dw,
+                        int64_t ld_dw, int64_t m, int64_t n, int64_t k, void* stream) {
+  if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
+  if (n % 128 || k % 128) return PURO_ERR_SHAPE;
+  if (n == 0 || k == 0) return PURO_OK;
+  int r;
+  if ((r = check_mat(dw, ld_dw, k, 2)) != PURO_OK) return r;
+  if (m > 0) {
+    if ((r = check_mat(qdyt, ld_qdyt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
+    if ((r = check_mat(sdyt, ld_sdyt, n, 1)) != PURO_OK) return r;
+    if ((r = check_mat(qxt, ld_qxt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
+    if ((r = check_mat(sxt, ld_sxt, k, 1)) != PURO_OK) return r;
+  }
+  GemmArgs g{qdyt, ld_qdyt, sdyt, ld_sdyt, qxt, ld_qxt, sxt, ld_sxt, true,
+             nullptr, 0, 0, dw, ld_dw, n, k, m};
+  return launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+int puro_fp8_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PURO_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, puro::g_status, sizeof(int)) != cudaSuccess) return PURO_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(puro::g_status, &zero, sizeof(int)) != cudaSuccess) return PURO_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ self-test
+
+namespace puro {
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);  // nothing ever arrives
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns);
+}
+}  // namespace puro
+
+extern "C" int puro_fp8_test_bounded_wait(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000) limit_ns = 1000;
+  if (limit_ns > 5000000000ll) limit_ns = 5000000000ll;
+  DeviceInfo* dev = nullptr;
+  int r = current_device(&dev);
+  if (r != PURO_OK) return r;
+  puro::bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      (uint64_t)limit_ns);
+  return launch_status();
+}

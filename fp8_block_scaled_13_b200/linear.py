@@ -1,0 +1,170 @@
+"""Torch-facing wrappers of the C ABI: allocate outputs with torch, pass device
+pointers and the current stream, raise on a non-zero status.  No arithmetic
+happens here; every step runs in libpuro_fp8.so.
+
+Layouts (see include/puro_fp8.h):
+  * FP8 codes are torch.uint8 tensors (view them as torch.float8_e4m3fn to
+    decode); UE8M0 scales are torch.uint8 bytes, scale = 2^(b - 127).
+  * Activation/gradient scales are group-major [groups, ld] with
+    ld = rows rounded up to 16; the valid part is [:, :rows].
+  * Transposed (COLWISE) codes are [cols, ld] with ld = rows rounded up to 16.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+
+def _round16(n: int) -> int:
+    return (n + 15) // 16 * 16
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != _lib.PURO_OK:
+        raise _lib.PuroError(status, where)
+
+
+def _require(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("%s must be a row-major 2-D tensor" % name)
+
+
+@dataclass
+class QuantAct:
+    """Result of quant_act.  rows/cols describe the BF16 input."""
+    rows: int
+    cols: int
+    q: torch.Tensor | None = None    # [rows, cols] u8
+    s: torch.Tensor | None = None    # [cols/128, ld_s] u8, group-major
+    qt: torch.Tensor | None = None   # [cols, ld_qt] u8, transposed codes
+    st: torch.Tensor | None = None   # [ceil(rows/128), ld_st] u8, group-major
+
+
+@dataclass
+class QuantWeight:
+    n: int
+    k: int
+    q: torch.Tensor                  # [n, k] u8
+    s: torch.Tensor                  # [n/128, k/128] u8
+    qt: torch.Tensor | None = None   # [k, n] u8
+
+
+def quant_act(x: torch.Tensor, layout: str = "both", out: QuantAct | None = None) -> QuantAct:
+    """1x128 quantization of an activation/gradient x [rows, cols] (BF16)."""
+    _require(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    flag = {"rowwise": _lib.PURO_ROWWISE, "colwise": _lib.PURO_COLWISE, "both": _lib.PURO_BOTH}[layout]
+    dev = x.device
+    if out is None:
+        out = QuantAct(rows, cols)
+        if flag & _lib.PURO_ROWWISE:
+            out.q = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+            out.s = torch.empty((cols // 128, _round16(rows)), dtype=torch.uint8, device=dev)
+        if flag & _lib.PURO_COLWISE:
+            out.qt = torch.empty((cols, _round16(rows)), dtype=torch.uint8, device=dev)
+            out.st = torch.empty(((rows + 127) // 128, _round16(cols)), dtype=torch.uint8, device=dev)
+    z = 0
+    st = _lib.puro_fp8_quant_act(
+        x.data_ptr(), rows, cols, x.stride(0), flag,
+        out.q.data_ptr() if out.q is not None else None, out.q.stride(0) if out.q is not None else z,
+        out.s.data_ptr() if out.s is not None else None, out.s.stride(0) if out.s is not None else z,
+        out.qt.data_ptr() if out.qt is not None else None, out.qt.stride(0) if out.qt is not None else z,
+        out.st.data_ptr() if out.st is not None else None, out.st.stride(0) if out.st is not None else z,
+        _stream())
+    _check(st, "puro_fp8_quant_act")
+    return out
+
+
+def quant_weight(w: torch.Tensor, transpose: bool = True, out: QuantWeight | None = None) -> QuantWeight:
+    """128x128 block quantization of a weight w [n, k] (BF16)."""
+    _require(w, torch.bfloat16, "w")
+    n, k = w.shape
+    dev = w.device
+    if out is None:
+        out = QuantWeight(
+            n, k,
+            torch.empty((n, k), dtype=torch.uint8, device=dev),
+            torch.empty((n // 128, k // 128), dtype=torch.uint8, device=dev),
+            torch.empty((k, n), dtype=torch.uint8, device=dev) if transpose else None)
+    st = _lib.puro_fp8_quant_weight(
+        w.data_ptr(), n, k, w.stride(0), out.q.data_ptr(), out.q.stride(0), out.s.data_ptr(),
+        out.qt.data_ptr() if out.qt is not None else None,
+        out.qt.stride(0) if out.qt is not None else 0, _stream())
+    _check(st, "puro_fp8_quant_weight")
+    return out
+
+
+def gemm_fprop(xq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T [m, n] BF16 from the ROWWISE quantization of X and the weight's."""
+    m, k, n = xq.rows, xq.cols, wq.n
+    if wq.k != k:
+        raise ValueError("inner dimensions differ: %d vs %d" % (k, wq.k))
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=xq.q.device)
+    st = _lib.puro_fp8_gemm_fprop(
+        xq.q.data_ptr(), xq.q.stride(0), xq.s.data_ptr(), xq.s.stride(0),
+        wq.q.data_ptr(), wq.q.stride(0), wq.s.data_ptr(),
+        out.data_ptr(), out.stride(0), m, n, k, _stream())
+    _check(st, "puro_fp8_gemm_fprop")
+    return out
+
+
+def gemm_dgrad(dyq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """dX = dY W [m, k] BF16 from the ROWWISE quantization of dY and W's transposed codes."""
+    m, n, k = dyq.rows, dyq.cols, wq.k
+    if wq.n != n:
+        raise ValueError("dY has %d columns, W has %d rows" % (n, wq.n))
+    if wq.qt is None:
+        raise ValueError("dgrad needs the transposed weight codes (quant_weight(transpose=True))")
+    if out is None:
+        out = torch.empty((m, k), dtype=torch.bfloat16, device=dyq.q.device)
+    st = _lib.puro_fp8_gemm_dgrad(
+        dyq.q.data_ptr(), dyq.q.stride(0), dyq.s.data_ptr(), dyq.s.stride(0),
+        wq.qt.data_ptr(), wq.qt.stride(0), wq.s.data_ptr(),
+        out.data_ptr(), out.stride(0), m, n, k, _stream())
+    _check(st, "puro_fp8_gemm_dgrad")
+    return out
+
+
+def gemm_wgrad(dyq: QuantAct, xq: QuantAct, out: torch.Tensor | None = None) -> torch.Tensor:
+    """dW = dY^T X [n, k] BF16 from the COLWISE quantizations of dY and X."""
+    m, n, k = dyq.rows, dyq.cols, xq.cols
+    if xq.rows != m:
+        raise ValueError("dY and X have different token counts")
+    if out is None:
+        out = torch.empty((n, k), dtype=torch.bfloat16, device=dyq.qt.device)
+    st = _lib.puro_fp8_gemm_wgrad(
+        dyq.qt.data_ptr(), dyq.qt.stride(0), dyq.st.data_ptr(), dyq.st.stride(0),
+        xq.qt.data_ptr(), xq.qt.stride(0), xq.st.data_ptr(), xq.st.stride(0),
+        out.data_ptr(), out.stride(0), m, n, k, _stream())
+    _check(st, "puro_fp8_gemm_wgrad")
+    return out
+
+
+def device_status() -> int:
+    """Synchronize the current stream and return/clear the device error word."""
+    return _lib.puro_fp8_device_status(_stream())
+
+
+def linear_forward(x: torch.Tensor, w: torch.Tensor):
+    """Quantize X and W, then Y = X W^T.  Returns (y, xq, wq)."""
+    xq = quant_act(x, "both")
+    wq = quant_weight(w, transpose=True)
+    return gemm_fprop(xq, wq), xq, wq
+
+
+def linear_backward(dy: torch.Tensor, xq: QuantAct, wq: QuantWeight):
+    """Quantize dY both ways, then dX = dY W and dW = dY^T X.  Returns (dx, dw)."""
+    dyq = quant_act(dy, "both")
+    return gemm_dgrad(dyq, wq), gemm_wgrad(dyq, xq)

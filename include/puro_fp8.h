@@ -1,0 +1,187 @@
+/*
+ * puro_fp8.h -- C ABI of the block-scaled FP8 linear layer for NVIDIA B200
+ * (sm_100a).
+ *
+ * The method (Puro-2B report; paper.rainbus.top summary, background
+ * "FP8 块级混合精度训练" and "方法步骤详情" step (3); ta-paperlens explainer
+ * §3.2; paperlayer.ai summary, Appendix C "FP8 implementation pipeline"):
+ * the fprop, dgrad and wgrad GEMMs of every transformer linear layer run in
+ * E4M3 FP8.  Activations and gradients carry one power-of-two scale per 128
+ * consecutive values along the GEMM reduction dimension, weights one per
+ * 128x128 block; scales are computed online from the BF16 tensor.  This
+ * library implements that hot path: the quantizers and the three GEMMs
+ * (FP32 accumulation, BF16 output).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer is a DEVICE pointer owned by the caller.  The library never
+ *    allocates or frees memory on a call.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream).  Nothing synchronizes the host except
+ *    puro_fp8_device_status().
+ *  - Errors are returned as puro_status codes; nothing throws or aborts.  An
+ *    argument error is detected on the host and returns before any launch.
+ *  - Element formats:
+ *      BF16   : IEEE binary32 upper half (torch.bfloat16).
+ *      E4M3   : OCP FP8 "FN" (torch.float8_e4m3fn): bias 7, max 448, NaN 0x7F
+ *               and 0xFF, no infinity.  Round to nearest even, saturating.
+ *      UE8M0  : one byte b per scale, scale = 2^(b - 127).  b = e + 127 where e
+ *               is the smallest integer with amax <= 448 * 2^e over the group,
+ *               clamped to [-127, 127]; an all-zero group has e = 0 (b = 127).
+ *               0xFF is never produced.
+ *  - Layouts are row-major; every leading dimension (`ld_*`) is in ELEMENTS of
+ *    the array it describes (bytes for the FP8 and UE8M0 arrays) and must make
+ *    each row start on a 16-byte boundary.  Every pointer must be 16-byte
+ *    aligned.
+ *  - Activation/gradient scale arrays are stored GROUP-MAJOR: for a quantized
+ *    matrix Q [rows, cols] grouped along cols, the scale of (row r, group g)
+ *    is s[g * ld_s + r].  This keeps the 128 scales of one GEMM tile
+ *    contiguous so the GEMM loads them with one bulk tensor copy.
+ *  - Weight scale arrays are compact row-major [n/128, k/128].
+ */
+#ifndef PURO_FP8_H
+#define PURO_FP8_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PURO_API __attribute__((visibility("default")))
+#else
+#define PURO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PURO_OK = 0,
+    PURO_ERR_NULL = -1,               /* a required pointer is NULL               */
+    PURO_ERR_ALIGN = -2,              /* pointer or leading dim not 16-B aligned   */
+    PURO_ERR_SHAPE = -3,              /* a size or leading dim is out of range     */
+    PURO_ERR_LAYOUT = -4,             /* unknown layout flag                       */
+    PURO_ERR_CUDA = -5,               /* a CUDA runtime/driver call failed         */
+    PURO_ERR_UNSUPPORTED_DEVICE = -6, /* current device is not sm_100              */
+    PURO_ERR_DEVICE_TIMEOUT = -7      /* a bounded on-device wait expired          */
+} puro_status;
+
+/* Layout flags of puro_fp8_quant_act. */
+enum {
+    PURO_ROWWISE = 1,  /* groups of 128 along cols, codes kept in place          */
+    PURO_COLWISE = 2,  /* groups of 128 along rows, codes written transposed     */
+    PURO_BOTH = 3      /* both outputs from one read of x                         */
+};
+
+/*
+ * puro_fp8_quant_act -- online 1x128 quantization of an activation or
+ * gradient (the "activations and gradients, one scale per 128 elements along
+ * the reduction direction" rule of ta-paperlens §3.2 and the 1-D groups of
+ * paper.rainbus.top step (3)).
+ *
+ * x      : BF16 [rows, cols], row stride ld_x elements (ld_x >= cols).
+ * layout : PURO_ROWWISE, PURO_COLWISE or PURO_BOTH.
+ *
+ * ROWWISE output (the fprop/dgrad operand: the reduction dim is cols):
+ *   cols % 128 == 0 is required.
+ *   q  : E4M3 [rows, cols], row stride ld_q bytes (ld_q >= cols).
+ *   s  : UE8M0 group-major [cols/128][ld_s], ld_s >= rows; scale of group
+ *        (r, g) = x[r, 128g .. 128g+127] at s[g*ld_s + r].
+ * COLWISE output (the wgrad operand: the reduction dim is rows = tokens):
+ *   qt : E4M3 [cols, ld_qt], ld_qt >= rows rounded up to 16; qt[c*ld_qt + r]
+ *        is the code of x[r, c].  Bytes [rows, round_up(rows,16)) of each row
+ *        are written as 0; bytes beyond are not touched.
+ *   st : UE8M0 group-major [ceil(rows/128)][ld_st], ld_st >= cols; the scale of
+ *        (column c, row group g) -- rows 128g .. min(128g+127, rows-1), the last
+ *        group may be short and only its valid rows enter the amax -- is at
+ *        st[g*ld_st + c].
+ * Unused outputs may be NULL.  rows == 0 or cols == 0 is a no-op.
+ * Limits: rows, cols < 2^31.
+ */
+PURO_API int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int layout,
+                       void* q, int64_t ld_q, void* s, int64_t ld_s,
+                       void* qt, int64_t ld_qt, void* st, int64_t ld_st,
+                       void* stream);
+
+/*
+ * puro_fp8_quant_weight -- 128x128 block quantization of a weight
+ * (paper.rainbus.top background and step (3): "weights in 128x128 blocks,
+ * one online power-of-two scale each").
+ *
+ * w  : BF16 [n, k], row stride ld_w elements; n % 128 == 0, k % 128 == 0.
+ * q  : E4M3 [n, k], row stride ld_q bytes.
+ * s  : UE8M0 [n/128, k/128] compact row-major; s[bn*(k/128) + bk].
+ * qt : optional (NULL to skip) E4M3 [k, n], row stride ld_qt bytes, the byte
+ *      transpose of q.  Because the blocks are square, block (bk, bn) of qt has
+ *      the scale s[bn*(k/128) + bk]; no second scale array exists.  This is the
+ *      K-contiguous weight operand of dgrad.
+ */
+PURO_API int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w,
+                          void* q, int64_t ld_q, void* s,
+                          void* qt, int64_t ld_qt, void* stream);
+
+/*
+ * puro_fp8_gemm_fprop -- Y = X W^T (forward GEMM of paperlayer.ai Appendix C).
+ *   Y[i,j] = sum_kb 2^(ex[i,kb] + ew[j/128,kb]) * sum_{k in kb} qx[i,k] qw[j,k]
+ * accumulated in FP32 on the tensor cores, rounded once to BF16 (RNE).
+ * qx : E4M3 [m, k] (ld_qx),  sx : group-major [k/128][ld_sx]  (quant_act ROWWISE of X)
+ * qw : E4M3 [n, k] (ld_qw),  sw : [n/128, k/128]              (quant_weight of W)
+ * y  : BF16 [m, n], row stride ld_y elements.
+ * k % 128 == 0, n % 128 == 0, k <= 32768; any m >= 0 (rows >= m are neither
+ * read nor written).
+ */
+PURO_API int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx, int64_t ld_sx,
+                        const void* qw, int64_t ld_qw, const void* sw,
+                        void* y, int64_t ld_y, int64_t m, int64_t n, int64_t k, void* stream);
+
+/*
+ * puro_fp8_gemm_dgrad -- dX = dY W (data-gradient GEMM, reduction over n).
+ * qdy : E4M3 [m, n] (ld_qdy), sdy : group-major [n/128][ld_sdy] (quant_act ROWWISE of dY)
+ * qwt : E4M3 [k, n] (ld_qwt)  -- the `qt` output of puro_fp8_quant_weight
+ * sw  : [n/128, k/128]        -- the same weight scale array as fprop
+ * dx  : BF16 [m, k], row stride ld_dx elements.
+ * k % 128 == 0, n % 128 == 0, n <= 32768; any m >= 0.
+ */
+PURO_API int puro_fp8_gemm_dgrad(const void* qdy, int64_t ld_qdy, const void* sdy, int64_t ld_sdy,
+                        const void* qwt, int64_t ld_qwt, const void* sw,
+                        void* dx, int64_t ld_dx, int64_t m, int64_t n, int64_t k, void* stream);
+
+/*
+ * puro_fp8_gemm_wgrad -- dW = dY^T X (weight-gradient GEMM, reduction over the
+ * m tokens, both operands quantized along m as ta-paperlens §3.2 prescribes
+ * for gradients and activations).
+ * qdyt : E4M3 [n, ld_qdyt], sdyt : group-major [ceil(m/128)][ld_sdyt] (COLWISE of dY)
+ * qxt  : E4M3 [k, ld_qxt],  sxt  : group-major [ceil(m/128)][ld_sxt]  (COLWISE of X)
+ * dw   : BF16 [n, k], row stride ld_dw elements.
+ * n % 128 == 0, k % 128 == 0; any m >= 0 (a short last token group is read with
+ * zero padding; m == 0 writes dW = 0).
+ */
+PURO_API int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* sdyt, int64_t ld_sdyt,
+                        const void* qxt, int64_t ld_qxt, const void* sxt, int64_t ld_sxt,
+                        void* dw, int64_t ld_dw, int64_t m, int64_t n, int64_t k, void* stream);
+
+/*
+ * puro_fp8_device_status -- synchronizes `stream`, then returns and clears the
+ * library's device error word for the current device: PURO_OK, or
+ * PURO_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the last
+ * call (that kernel's output is then undefined), or PURO_ERR_CUDA if the
+ * synchronization itself failed.
+ */
+PURO_API int puro_fp8_device_status(void* stream);
+
+/* Human-readable name of a puro_status code (static storage). */
+PURO_API const char* puro_fp8_status_string(int status);
+
+/*
+ * puro_fp8_test_bounded_wait -- self-test of the bounded-wait machinery: launches
+ * one block that waits on a shared-memory barrier nothing will ever arrive on,
+ * with a limit of `limit_ns` nanoseconds (clamped to [1e3, 5e9]).  The wait
+ * must give up, record PURO_ERR_DEVICE_TIMEOUT in the device error word and
+ * return; puro_fp8_device_status() then reports it.  Nothing faults or traps.
+ */
+PURO_API int puro_fp8_test_bounded_wait(int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PURO_FP8_H */

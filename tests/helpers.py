@@ -1,0 +1,52 @@
+"""Shared helpers of the GPU parity tests (comparison and tolerance logic)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+
+def np_u8(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def gpu_rowwise(xq, rows=None):
+    """(q [R,C], s [R,G]) in the oracle's orientation from a QuantAct."""
+    R = xq.rows
+    q = np_u8(xq.q)
+    s = np_u8(xq.s)[:, :R].T
+    if rows is not None:
+        q, s = q[rows], s[rows]
+    return q, s
+
+
+def gpu_colwise(xq):
+    """(qt [C,R], st [C,G]) in the oracle's orientation, plus the zero padding."""
+    R, C = xq.rows, xq.cols
+    qt_full = np_u8(xq.qt)
+    st = np_u8(xq.st)[:, :C].T
+    pad = qt_full[:, R:(R + 15) // 16 * 16]
+    return qt_full[:, :R], st, pad
+
+
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 7)
+
+
+def gemm_errors(got: torch.Tensor, ref64: np.ndarray, oracle):
+    """Relative Frobenius error against the oracle's BF16-rounded result, and
+    the worst excess of |got - ref| over 4e-3*rms(ref) + 1 BF16 ulp(ref)."""
+    g = got.detach().float().cpu().numpy().astype(np.float64)
+    ref_bf16 = oracle.bf16_to_double(oracle.to_bf16_bits(ref64))
+    den = np.linalg.norm(ref_bf16)
+    rel = np.linalg.norm(g - ref_bf16) / den if den > 0 else np.linalg.norm(g)
+    rms = np.sqrt(np.mean(ref64 ** 2)) if ref64.size else 0.0
+    excess = np.abs(g - ref64) - (4e-3 * rms + bf16_ulp(ref64))
+    return float(rel), float(excess.max()) if excess.size else -1.0
+
+
+def assert_gemm_close(got, ref64, oracle, what=""):
+    rel, excess = gemm_errors(got, ref64, oracle)
+    assert rel <= 1e-3, "%s: relative Frobenius error %.3g > 1e-3" % (what, rel)
+    assert excess <= 0.0, "%s: an element exceeds 4e-3*rms + 1 ulp by %.3g" % (what, excess)
+    return rel

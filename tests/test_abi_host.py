@@ -1,0 +1,156 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/puro_fp8.h declares, and rejects bad arguments
+before touching CUDA.  Also checks that the product code never imports the
+oracle."""
+import ast
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "puro_fp8.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_block_scaled_13_b200 import build, _lib
+    build.build()
+    return _lib
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"PURO_API\s+(?:const\s+)?\w+\*?\s+\*?(puro_fp8_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_abi():
+    names = _declared()
+    for must in ("puro_fp8_quant_act", "puro_fp8_quant_weight", "puro_fp8_gemm_fprop",
+                 "puro_fp8_gemm_dgrad", "puro_fp8_gemm_wgrad", "puro_fp8_device_status",
+                 "puro_fp8_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (\w+)", out))
+    assert set(_declared()) <= exported
+    # nothing else leaks out (the static CUDA runtime stays hidden)
+    assert {s for s in exported if not s.startswith("puro_fp8_")} <= {"_init", "_fini"}
+    assert set(lib.EXPORTS) == set(_declared())
+
+
+def test_status_strings(lib):
+    for code in range(0, -8, -1):
+        s = lib.status_string(code)
+        assert s.startswith("PURO_")
+    assert "unknown" in lib.status_string(-99)
+
+
+A = 1 << 20  # a 16-byte-aligned fake device address; never dereferenced here
+
+
+@pytest.mark.parametrize("args,code", [
+    # bad layout flag
+    ((A, 16, 128, 128, 7, A, 128, A, 16, None, 0, None, 0), -4),
+    # cols not a multiple of 128
+    ((A, 16, 100, 128, 1, A, 128, A, 16, None, 0, None, 0), -3),
+    # negative rows
+    ((A, -1, 128, 128, 1, A, 128, A, 16, None, 0, None, 0), -3),
+    # null input
+    ((None, 16, 128, 128, 1, A, 128, A, 16, None, 0, None, 0), -1),
+    # misaligned input pointer
+    ((A + 2, 16, 128, 128, 1, A, 128, A, 16, None, 0, None, 0), -2),
+    # ld_x < cols
+    ((A, 16, 256, 128, 1, A, 256, A, 16, None, 0, None, 0), -3),
+    # ROWWISE without q
+    ((A, 16, 128, 128, 1, None, 128, A, 16, None, 0, None, 0), -1),
+    # scale leading dim < rows
+    ((A, 32, 128, 128, 1, A, 128, A, 16, None, 0, None, 0), -3),
+    # scale leading dim not a multiple of 16
+    ((A, 17, 128, 128, 1, A, 128, A, 24, None, 0, None, 0), -2),
+    # COLWISE: qt leading dim below rows rounded to 16
+    ((A, 17, 128, 128, 2, None, 0, None, 0, A, 16, A, 128), -3),
+    # COLWISE: missing st
+    ((A, 16, 128, 128, 2, None, 0, None, 0, A, 16, None, 128), -1),
+])
+def test_quant_act_argument_errors(lib, args, code):
+    assert lib.puro_fp8_quant_act(*args, None) == code
+
+
+def test_quant_act_empty_is_noop(lib):
+    assert lib.puro_fp8_quant_act(None, 0, 128, 128, 3, None, 0, None, 0, None, 0, None, 0, None) == 0
+    assert lib.puro_fp8_quant_act(None, 5, 0, 0, 3, None, 0, None, 0, None, 0, None, 0, None) == 0
+
+
+@pytest.mark.parametrize("args,code", [
+    ((A, 100, 128, 128, A, 128, A, None, 0), -3),       # n not multiple of 128
+    ((A, 128, 100, 128, A, 128, A, None, 0), -3),       # k not multiple of 128
+    ((A, 128, 128, 128, None, 128, A, None, 0), -1),    # q null
+    ((A, 128, 128, 128, A, 128, None, None, 0), -1),    # s null
+    ((A, 128, 128, 128, A, 128, A, A, 64), -3),         # ld_qt < n
+    ((A, 128, 128, 128, A + 8, 128, A, None, 0), -2),   # misaligned q
+])
+def test_quant_weight_argument_errors(lib, args, code):
+    assert lib.puro_fp8_quant_weight(*args, None) == code
+
+
+@pytest.mark.parametrize("fn,args,code", [
+    ("fprop", (A, 256, A, 64, A, 256, A, A, 320, 64, 320, 256), -3),    # n % 128
+    ("fprop", (A, 256, A, 64, A, 256, A, A, 256, 64, 256, 200), -3),    # k % 128
+    ("fprop", (A, 256, A, 64, A, 256, A, A, 256, 64, 256, 65536), -3),  # k > 32768
+    ("fprop", (A, 256, A, 60, A, 256, A, A, 256, 64, 256, 256), -3),    # ld_sx < m
+    ("fprop", (A, 256, A, 64, A, 256, None, A, 256, 64, 256, 256), -1), # sw null
+    ("fprop", (A, 256, A, 64, A, 256, A, A, 100, 64, 256, 256), -3),    # ld_y < n
+    ("fprop", (A, 256, A, 64, A, 256, A, A + 4, 256, 64, 256, 256), -2),
+    ("dgrad", (A, 256, A, 64, A, 256, A, A, 256, 64, 256, 256), 0),     # placeholder (valid)
+    ("dgrad", (A, 128, A, 64, A, 256, A, A, 256, 64, 256, 256), -3),    # ld_qdy < n
+    ("wgrad", (A, 64, A, 256, A, 64, A, 256, A, 256, 64, 256, 256), 0), # placeholder (valid)
+    ("wgrad", (A, 48, A, 256, A, 64, A, 256, A, 256, 64, 256, 256), -3),  # ld_qdyt < m
+    ("wgrad", (A, 64, A, 256, A, 64, A, 256, A, 256, 64, 200, 256), -3),  # n % 128
+])
+def test_gemm_argument_errors(lib, fn, args, code):
+    f = getattr(lib, "puro_fp8_gemm_" + fn)
+    if code == 0:
+        pytest.skip("valid arguments need a device")
+    assert f(*args, None) == code
+
+
+def test_gemm_empty_is_noop(lib):
+    assert lib.puro_fp8_gemm_fprop(None, 0, None, 0, None, 0, None, None, 0, 0, 256, 256, None) == 0
+    assert lib.puro_fp8_gemm_wgrad(None, 0, None, 0, None, 0, None, 0, None, 0, 64, 0, 256, None) == 0
+
+
+def _imports(path):
+    tree = ast.parse(open(path).read())
+    mods = set()
+    for node in ast.walk(tree):
+        if isinstance(node, ast.Import):
+            mods |= {a.name.split(".")[0] for a in node.names}
+        elif isinstance(node, ast.ImportFrom) and node.module and node.level == 0:
+            mods.add(node.module.split(".")[0])
+    return mods
+
+
+def test_product_never_imports_oracle():
+    pkg = os.path.join(ROOT, "fp8_block_scaled_13_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith(".py"):
+                assert "oracle" not in _imports(os.path.join(dirpath, f)), f
+            if f.endswith((".cu", ".cuh", ".h", ".c", ".cpp")):
+                assert "puro_oracle" not in open(os.path.join(dirpath, f)).read(), f
+
+
+def test_oracle_never_imports_product():
+    odir = os.path.join(ROOT, "oracle")
+    for f in os.listdir(odir):
+        if f.endswith(".py"):
+            assert "fp8_block_scaled_13_b200" not in _imports(os.path.join(odir, f))
+        if f.endswith(".c"):
+            src = open(os.path.join(odir, f)).read()
+            includes = re.findall(r'#include\s*[<"]([^>"]+)', src)
+            assert not any("puro_fp8" in h or h.startswith("cuda") for h in includes), includes

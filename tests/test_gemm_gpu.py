@@ -1,0 +1,116 @@
+"""GPU fprop/dgrad/wgrad vs the FP64 oracle.
+
+Tolerance (block-scaled FP8 linear layer spec): relative Frobenius error
+<= 1e-3 against the oracle's result rounded to BF16, and every element within
+4e-3 * rms(Y_ref) + 1 BF16 ulp(Y_ref) of the unrounded FP64 result.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_gemm_close, gpu_colwise, gpu_rowwise
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    import fp8_block_scaled_13_b200 as m
+    from fp8_block_scaled_13_b200 import build
+    build.build()
+    return m
+
+
+def _layer(m, n, k, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(m, k, generator=g).to(torch.bfloat16)
+    w = (torch.randn(n, k, generator=g) * 0.02).to(torch.bfloat16)
+    dy = (torch.randn(m, n, generator=g) * 1e-3).to(torch.bfloat16)
+    return x, w, dy
+
+
+def _run(fp8, x, w, dy):
+    dev = torch.device("cuda")
+    y, xq, wq = fp8.linear_forward(x.to(dev), w.to(dev))
+    dx, dw = fp8.linear_backward(dy.to(dev), xq, wq)
+    torch.cuda.synchronize()
+    assert fp8.device_status() == 0
+    return y, dx, dw
+
+
+@pytest.mark.parametrize("m,n,k", [
+    (256, 384, 512),     # the single-fprop workload's shape
+    (300, 384, 512),     # ragged token count
+    (1, 128, 128),       # degenerate: one token, one block
+    (129, 256, 384),
+    (520, 640, 256),     # N not a multiple of the 256-wide tile
+    (64, 128, 1024),
+])
+def test_linear_layer_small(fp8, oracle_mod, m, n, k):
+    x, w, dy = _layer(m, n, k, m + n + k)
+    y, dx, dw = _run(fp8, x, w, dy)
+    assert_gemm_close(y, oracle_mod.linear_fprop(x, w), oracle_mod, "fprop")
+    assert_gemm_close(dx, oracle_mod.linear_dgrad(dy, w), oracle_mod, "dgrad")
+    assert_gemm_close(dw, oracle_mod.linear_wgrad(dy, x), oracle_mod, "wgrad")
+
+
+def test_identity_weight_exact(fp8, oracle_mod):
+    """W = I: Y equals the dequantized X exactly (each product has <= 4
+    significant bits, so FP32 accumulation and BF16 rounding are exact)."""
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(200, 256, generator=g) * 3).to(torch.bfloat16)
+    w = torch.eye(256, dtype=torch.bfloat16)
+    y, xq, wq = fp8.linear_forward(x.cuda(), w.cuda())
+    torch.cuda.synchronize()
+    ref = oracle_mod.linear_fprop(x, w)
+    got = y.float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(got, ref)
+    # dgrad with W = I is exact as well
+    dx = fp8.gemm_dgrad(fp8.quant_act(x.cuda(), "rowwise"), wq)
+    torch.cuda.synchronize()
+    assert np.array_equal(dx.float().cpu().numpy().astype(np.float64), ref)
+
+
+def test_permutation_and_power_of_two_exact(fp8, oracle_mod):
+    """A permutation weight and power-of-two activations: exact results."""
+    g = torch.Generator().manual_seed(6)
+    perm = torch.randperm(384, generator=g)
+    w = torch.zeros(384, 384)
+    w[torch.arange(384), perm] = 1.0
+    x = torch.exp2(torch.randint(-6, 6, (130, 384), generator=g).float()) * \
+        torch.where(torch.rand(130, 384, generator=g) < 0.5, -1.0, 1.0)
+    x, w = x.to(torch.bfloat16), w.to(torch.bfloat16)
+    y, _, _ = fp8.linear_forward(x.cuda(), w.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(y.float().cpu().numpy().astype(np.float64), oracle_mod.linear_fprop(x, w))
+
+
+def test_all_ones_closed_form(fp8):
+    x = torch.ones(70, 512, dtype=torch.bfloat16, device="cuda")
+    w = torch.ones(256, 512, dtype=torch.bfloat16, device="cuda")
+    y, _, _ = fp8.linear_forward(x, w)
+    torch.cuda.synchronize()
+    assert torch.all(y == 512.0)
+
+
+def test_zero_tokens_wgrad_is_zero(fp8):
+    x = torch.zeros(0, 256, dtype=torch.bfloat16, device="cuda")
+    dy = torch.zeros(0, 128, dtype=torch.bfloat16, device="cuda")
+    xq = fp8.quant_act(x, "both")
+    dyq = fp8.quant_act(dy, "both")
+    dw = torch.full((128, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    fp8.gemm_wgrad(dyq, xq, out=dw)
+    torch.cuda.synchronize()
+    assert torch.all(dw == 0)
+
+
+def test_output_strides(fp8, oracle_mod):
+    """Outputs written into a column slice of a wider buffer leave the rest alone."""
+    x, w, _ = _layer(136, 256, 256, 9)
+    xq = fp8.quant_act(x.cuda(), "rowwise")
+    wq = fp8.quant_weight(w.cuda())
+    buf = torch.full((136, 512), -1.0, dtype=torch.bfloat16, device="cuda")
+    fp8.gemm_fprop(xq, wq, out=buf[:, 128:384])
+    torch.cuda.synchronize()
+    assert torch.all(buf[:, :128] == -1) and torch.all(buf[:, 384:] == -1)
+    assert_gemm_close(buf[:, 128:384], oracle_mod.linear_fprop(x, w), oracle_mod, "strided fprop")

@@ -1,0 +1,137 @@
+"""GPU quantizers vs the CPU oracle: codes and scale bytes must match bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import gpu_colwise, gpu_rowwise, np_u8
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    import fp8_block_scaled_13_b200 as m
+    from fp8_block_scaled_13_b200 import build
+    build.build()
+    return m
+
+
+def _rand(shape, seed, lo=-20, hi=20):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(*shape, generator=g) * torch.exp2(
+        torch.randint(lo, hi, shape, generator=g).float())
+    return x.to(torch.bfloat16)
+
+
+def _check_all(fp8, oracle_mod, x, layout="both"):
+    xq = fp8.quant_act(x.cuda(), layout)
+    torch.cuda.synchronize()
+    assert fp8.device_status() == 0
+    if xq.q is not None:
+        q, s = gpu_rowwise(xq)
+        oq, os_ = oracle_mod.quant_rowwise(x)
+        assert np.array_equal(s, os_), "rowwise scales differ"
+        assert np.array_equal(q, oq), "rowwise codes differ at %s" % (np.argwhere(q != oq)[:5],)
+    if xq.qt is not None:
+        qt, st, pad = gpu_colwise(xq)
+        oqt, ost = oracle_mod.quant_colwise(x)
+        assert np.array_equal(st, ost), "colwise scales differ"
+        assert np.array_equal(qt, oqt), "colwise codes differ at %s" % (np.argwhere(qt != oqt)[:5],)
+        assert not pad.any(), "padding of the transposed codes is not zero"
+    return xq
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (300, 384), (128, 1024), (257, 256), (1000, 640)])
+@pytest.mark.parametrize("layout", ["rowwise", "colwise", "both"])
+def test_quant_act_random(fp8, oracle_mod, rows, cols, layout):
+    _check_all(fp8, oracle_mod, _rand((rows, cols), rows * 7 + cols), layout)
+
+
+def test_quant_act_every_bf16_pattern(fp8, oracle_mod):
+    """Every finite BF16 value appears once as an element (510 rows x 128)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    bits = bits[((bits >> 7) & 0xFF) != 0xFF]
+    assert bits.size == 510 * 128
+    rng = np.random.default_rng(0)
+    rng.shuffle(bits)
+    x = torch.from_numpy(bits.view(np.int16).reshape(510, 128).copy()).view(torch.bfloat16)
+    _check_all(fp8, oracle_mod, x, "both")
+    # and sorted, so that each group spans a narrow range of magnitudes
+    xs = torch.from_numpy(np.sort(bits).view(np.int16).reshape(510, 128).copy()).view(torch.bfloat16)
+    _check_all(fp8, oracle_mod, xs, "both")
+
+
+def test_quant_act_adversarial_groups(fp8, oracle_mod):
+    x = _rand((256, 1280), 11).float()
+    x[0, 0:128] = 0.0                                  # all-zero group
+    x[1, 0:128] = -0.0                                 # negative zeros
+    x[2, 0:128] = torch.linspace(-1, 1, 128) * 2.0 ** -130   # subnormal-only
+    x[3, 0:128] = 1e-3
+    x[3, 5] = 448.0                                    # amax exactly 448
+    x[4, 0:128] = 1e-3
+    x[4, 9] = -450.0                                   # next BF16 above 448
+    for kk, k in enumerate(range(-10, 10, 4)):
+        x[5 + kk, 128:256] = 0.5
+        x[5 + kk, 130] = 448.0 * 2.0 ** k              # amax = 448 * 2^k
+        x[5 + kk, 256:384] = 0.5
+        x[5 + kk, 300] = 450.0 * 2.0 ** k              # just above it
+    x[20, 384:512] = 1.0
+    x[20, 400] = 3.0e38                                # near BF16 max
+    x[21, 512:640] = torch.arange(128) * 2.0 ** -133   # smallest subnormals
+    x[22:150, 640:768] = 0.0                           # a zero 128-row band (colwise zero group)
+    x[30, 768:896] = 224.0                             # half of 448: exponent boundary
+    x[31, 768:896] = 1.75                              # 1.75 = 448 * 2^-8
+    x[32, 768:896] = 1.78125
+    _check_all(fp8, oracle_mod, x.to(torch.bfloat16), "both")
+
+
+def test_quant_act_strided_input(fp8, oracle_mod):
+    """A column slice of a wider tensor (ld_x > cols) and rows not multiple of 16."""
+    base = _rand((200, 768), 12)
+    xv = base.cuda()[:, 128:512]
+    assert xv.stride(0) == 768
+    xq = fp8.quant_act(xv, "both")
+    torch.cuda.synchronize()
+    x = base[:, 128:512].contiguous()
+    q, s = gpu_rowwise(xq)
+    oq, os_ = oracle_mod.quant_rowwise(x)
+    assert np.array_equal(q, oq) and np.array_equal(s, os_)
+    qt, st, pad = gpu_colwise(xq)
+    oqt, ost = oracle_mod.quant_colwise(x)
+    assert np.array_equal(qt, oqt) and np.array_equal(st, ost) and not pad.any()
+
+
+@pytest.mark.parametrize("n,k", [(128, 128), (384, 512), (3072, 2048), (2048, 6144)])
+def test_quant_weight(fp8, oracle_mod, n, k):
+    g = torch.Generator().manual_seed(n + k)
+    w = (torch.randn(n, k, generator=g) * 0.02).to(torch.bfloat16)
+    w[:128, :128] = 0   # a zero block
+    wq = fp8.quant_weight(w.cuda(), transpose=True)
+    torch.cuda.synchronize()
+    oq, os_ = oracle_mod.quant_weight(w)
+    assert np.array_equal(np_u8(wq.s), os_)
+    assert np.array_equal(np_u8(wq.q), oq)
+    assert np.array_equal(np_u8(wq.qt), oq.T)
+
+
+def test_quant_weight_heavy_tails(fp8, oracle_mod):
+    w = _rand((256, 384), 13, -30, 30)
+    wq = fp8.quant_weight(w.cuda(), transpose=False)
+    torch.cuda.synchronize()
+    oq, os_ = oracle_mod.quant_weight(w)
+    assert np.array_equal(np_u8(wq.s), os_) and np.array_equal(np_u8(wq.q), oq)
+    assert wq.qt is None
+
+
+def test_bounded_wait_reports_timeout(fp8):
+    """A wait that can never complete gives up, records the timeout and returns."""
+    from fp8_block_scaled_13_b200 import _lib
+    assert fp8.device_status() == 0
+    st = _lib.puro_fp8_test_bounded_wait(20_000_000, torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    assert fp8.device_status() == _lib.PURO_ERR_DEVICE_TIMEOUT
+    assert fp8.device_status() == 0   # cleared by the read
+    # the context is still usable
+    x = _rand((128, 128), 14).cuda()
+    fp8.quant_act(x, "rowwise")
+    torch.cuda.synchronize()

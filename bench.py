@@ -1,0 +1,445 @@
+"""Benchmark of the block-scaled FP8 linear layer hot path on B200.
+
+One step = the whole hot path over one batch of the attention-projection
+workload (M = 8192 tokens, hidden 2048; the fused QKV projection 2048->3072
+and the output projection 2048->2048), for each of the two layers:
+  quant_weight(W) (+ transposed codes), quant_act(X, both), fprop,
+  quant_act(dY, both), dgrad, wgrad.
+value = GEMM FLOPs of the step (2*M*N*K per GEMM, three GEMMs per layer)
+divided by the device time of the whole step (quantizers included).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+With N > 1 (torchrun) every rank runs its own batch (data-parallel replicas,
+weak scaling); there is no collective in the step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "FP8 block-scaled GEMM TFLOP/s (fprop/dgrad/wgrad) and % of B200 FP8 peak"
+WORKLOAD = "attn_proj_m8192_h2048_qkv3072_o2048"
+SEED = 1
+M_TOKENS = 8192
+# dram__bytes_read.sum + dram__bytes_write.sum of one GEMM launch (fprop, QKV
+# layer) from the ncu capture summarised in profiles/; None until captured
+# for the current kernel.
+GEMM_TRAFFIC_BYTES = None
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def _parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- our arm
+
+class Step:
+    """Device buffers of one step and the launch sequence, with an event pair
+    around every launch (on the launching stream)."""
+
+    def __init__(self, wl, dev, n_sets=3):
+        import torch
+        import fp8_block_scaled_13_b200 as fp8
+        self.fp8 = fp8
+        self.torch = torch
+        self.layers = wl.layers
+        # rotating input sets: each set is larger than L2 in total
+        self.sets = []
+        for _ in range(n_sets):
+            self.sets.append([(L.x.to(dev), L.w.to(dev), L.dy.to(dev)) for L in wl.layers])
+        # outputs, allocated once and reused
+        self.out = []
+        for (x, w, dy) in self.sets[0]:
+            xq = fp8.quant_act(x, "both")
+            wq = fp8.quant_weight(w, transpose=True)
+            dyq = fp8.quant_act(dy, "both")
+            y = torch.empty((x.shape[0], w.shape[0]), dtype=torch.bfloat16, device=dev)
+            dx = torch.empty_like(x)
+            dw = torch.empty_like(w)
+            self.out.append((xq, wq, dyq, y, dx, dw))
+        torch.cuda.synchronize()
+        self.names = []
+        for L in wl.layers:
+            self.names += ["%s.quant_weight" % L.name, "%s.quant_x" % L.name, "%s.fprop" % L.name,
+                           "%s.quant_dy" % L.name, "%s.dgrad" % L.name, "%s.wgrad" % L.name]
+        self.launches_per_step = len(self.names)
+
+    def run(self, set_idx, events=None):
+        fp8 = self.fp8
+        ev = iter(events) if events is not None else None
+
+        def mark():
+            if ev is not None:
+                next(ev).record()
+
+        for (x, w, dy), (xq, wq, dyq, y, dx, dw) in zip(self.sets[set_idx], self.out):
+            mark(); fp8.quant_weight(w, transpose=True, out=wq); mark()
+            mark(); fp8.quant_act(x, "both", out=xq); mark()
+            mark(); fp8.gemm_fprop(xq, wq, out=y); mark()
+            mark(); fp8.quant_act(dy, "both", out=dyq); mark()
+            mark(); fp8.gemm_dgrad(dyq, wq, out=dx); mark()
+            mark(); fp8.gemm_wgrad(dyq, xq, out=dw); mark()
+
+
+def _unit_costs(wl):
+    """Algorithmic work per launch: FLOPs for the GEMMs, bytes for quantizers."""
+    costs = {}
+    for L in wl.layers:
+        m, n, k = L.m, L.n, L.k
+        costs["%s.quant_weight" % L.name] = ("bytes", n * k * 2 + 2 * n * k + (n // 128) * (k // 128))
+        costs["%s.quant_x" % L.name] = ("bytes", m * k * 2 + 2 * m * k + 2 * m * k // 128)
+        costs["%s.quant_dy" % L.name] = ("bytes", m * n * 2 + 2 * m * n + 2 * m * n // 128)
+        for g in ("fprop", "dgrad", "wgrad"):
+            costs["%s.%s" % (L.name, g)] = ("flops", 2 * m * n * k)
+    return costs
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from fp8_block_scaled_13_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    wl = inputs.attn_proj(seed=SEED + rank, m=M_TOKENS)
+    step = Step(wl, dev)
+    costs = _unit_costs(wl)
+    gemm_flops = wl.gemm_flops()
+    stream = torch.cuda.current_stream()
+
+    for i in range(args.warmup):
+        step.run(i % len(step.sets))
+    torch.cuda.synchronize()
+    status = step.fp8.device_status()
+    if status != 0:
+        raise RuntimeError("device status %d after warm-up" % status)
+
+    K = args.steps
+    nl = step.launches_per_step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl)] for _ in range(K)]
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(K):
+            step_ev[i][0].record(stream)
+            step.run(i % len(step.sets), ev[i])
+            step_ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    status = step.fp8.device_status()
+    if status != 0:
+        raise RuntimeError("device status %d in the timed region" % status)
+    clocks = clk.summary()
+
+    total_ms = t_start.elapsed_time(t_end)
+    per_launch = {name: [] for name in step.names}
+    for i in range(K):
+        for j, name in enumerate(step.names):
+            per_launch[name].append(ev[i][2 * j].elapsed_time(ev[i][2 * j + 1]))
+    ms_per_step = total_ms / K
+    if world > 1:
+        t = torch.tensor([ms_per_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_per_step = float(t.item())
+
+    peaks, peak_kind = _peaks()
+    fp8_peak_tf = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    value = gemm_flops * world / (ms_per_step * 1e-3) / 1e12
+
+    gemm_ms = sum(statistics.mean(per_launch[n]) for n in step.names if costs[n][0] == "flops")
+    gemm_tf = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    quant_ms = sum(statistics.mean(per_launch[n]) for n in step.names if costs[n][0] == "bytes")
+    quant_bytes = sum(costs[n][1] for n in step.names if costs[n][0] == "bytes")
+    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    breakdown = {}
+    for n in step.names:
+        kind, amount = costs[n]
+        ms = statistics.mean(per_launch[n])
+        rate = amount / (ms * 1e-3) / (1e12 if kind == "flops" else 1e9)
+        breakdown[n] = {"ms": round(ms, 5), ("tflops" if kind == "flops" else "gbs"): round(rate, 1)}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(wl, dev, K=min(K, 10), warmup=2)
+        if world > 1:
+            t = torch.tensor([e2e["ms_per_step"]], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e["ms_per_step"] = float(t.item())
+        e2e["value"] = round(gemm_flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12, 2)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, budget_s=15.0)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "e4m3",
+            "data": "synthetic",
+            "config": {
+                "workload": WORKLOAD,
+                "tokens_per_gpu": M_TOKENS, "hidden": 2048, "qkv_out": 3072, "o_out": 2048,
+                "seed": SEED,
+                "global_batch_tokens": M_TOKENS * world,
+                "l2": "3 rotating input sets of 132 MB each (> 126 MB L2)",
+                "parallelism": "dp%d replicas, no collective" % world,
+                "step": "per layer: quant_weight, quant_act(X), fprop, quant_act(dY), dgrad, wgrad",
+            },
+            "pct_fp8_peak": round(100.0 * value / world / fp8_peak_tf, 1),
+            "roofline": {
+                "bound": "tensor",
+                "kernel": "gemm_block_scaled_kernel (fprop/dgrad/wgrad, FLOP-weighted)",
+                "achieved": round(gemm_tf, 1),
+                "peak": round(fp8_peak_tf, 1),
+                "unit": "TFLOP/s",
+                "frac": round(gemm_tf / fp8_peak_tf, 4),
+                "peak_source": "%s: 2 x bf16_tflops_sustained (FP8 = 2 x BF16 nominal ratio)" % peak_kind,
+                "traffic": GEMM_TRAFFIC_BYTES,
+            },
+            "quantizers": {
+                "bound": "hbm", "achieved": round(quant_gbs, 1), "unit": "GB/s",
+                "peak": peaks["hbm_gbs"], "frac": round(quant_gbs / peaks["hbm_gbs"], 4),
+            },
+            "kernels": breakdown,
+            "gpu_launches": step.launches_per_step * K,
+            "clocks": clocks,
+            "wall_ms_timed_region": round(total_ms, 3),
+        }
+        if e2e is not None:
+            line["e2e"] = {"value": e2e["value"], "unit": "TFLOP/s",
+                           "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                           "ms_per_step": round(e2e["ms_per_step"], 3)}
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(wl, dev, K, warmup):
+    """Same step through the public API with pinned host inputs/outputs: every
+    step copies X, W, dY in and Y, dX, dW out inside the timed region."""
+    import torch
+    import fp8_block_scaled_13_b200 as fp8
+
+    host_in = [(L.x.pin_memory(), L.w.pin_memory(), L.dy.pin_memory()) for L in wl.layers]
+    host_out = [(torch.empty((L.m, L.n), dtype=torch.bfloat16).pin_memory(),
+                 torch.empty((L.m, L.k), dtype=torch.bfloat16).pin_memory(),
+                 torch.empty((L.n, L.k), dtype=torch.bfloat16).pin_memory()) for L in wl.layers]
+    h2d = sum(t.numel() * t.element_size() for tup in host_in for t in tup)
+    d2h = sum(t.numel() * t.element_size() for tup in host_out for t in tup)
+
+    def one():
+        for (hx, hw, hdy), (hy, hdx, hdw) in zip(host_in, host_out):
+            x = hx.to(dev, non_blocking=True)
+            w = hw.to(dev, non_blocking=True)
+            dy = hdy.to(dev, non_blocking=True)
+            y, xq, wq = fp8.linear_forward(x, w)
+            dx, dw = fp8.linear_backward(dy, xq, wq)
+            hy.copy_(y, non_blocking=True)
+            hdx.copy_(dx, non_blocking=True)
+            hdw.copy_(dw, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    return {"ms_per_step": s.elapsed_time(e) / K, "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def _oracle_sample(wl, rows_per_gemm):
+    """The hot path on a bounded sample, through the CPU oracle: for every
+    layer, `rows_per_gemm` output rows of fprop, dgrad and wgrad, including the
+    quantization those rows need.  Returns the sampled GEMM FLOPs."""
+    import numpy as np
+    import oracle
+
+    flops = 0
+    for L in wl.layers:
+        m, n, k = L.m, L.n, L.k
+        r = rows_per_gemm
+        rows = np.linspace(0, m - 1, r).astype(np.int64)
+        oracle.linear_fprop(L.x[rows], L.w)
+        oracle.linear_dgrad(L.dy[rows], L.w)
+        cols = np.linspace(0, n - 1, r).astype(np.int64)
+        oracle.linear_wgrad(L.dy[:, cols].contiguous(), L.x)
+        flops += 3 * 2 * r * n * k
+    return flops
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    n_cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    f = _oracle_sample(wl, 4)
+    dt = time.perf_counter() - t0
+    rows = max(4, min(1024, int(4 * budget_s / max(dt, 1e-3))))
+    t0 = time.perf_counter()
+    f = _oracle_sample(wl, rows)
+    dt = time.perf_counter() - t0
+    return {"value": round(f / dt / 1e12, 6), "unit": "TFLOP/s", "cores": n_cores,
+            "kind": "oracle",
+            "sample": "%d output rows of each of the 6 GEMMs (fprop/dgrad/wgrad x 2 layers) "
+                      "with the quantization they need, FP64 C oracle, %.1f s" % (rows, dt)}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle as it stands, on a bounded sample of the
+    same workload per step; rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from fp8_block_scaled_13_b200 import inputs
+    wl = inputs.attn_proj(seed=SEED, m=M_TOKENS)
+    rows = 8
+    for _ in range(args.warmup):
+        _oracle_sample(wl, rows)
+    t0 = time.perf_counter()
+    flops = 0
+    for _ in range(args.steps):
+        flops += _oracle_sample(wl, rows)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    n_cores = len(os.sched_getaffinity(0))
+    sample = ("%d output rows of each of the 6 GEMMs per step (fprop/dgrad/wgrad x 2 layers) "
+              "with the quantization they need, FP64 C oracle" % rows)
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "tokens_per_gpu": M_TOKENS, "hidden": 2048,
+                   "qkv_out": 3072, "o_out": 2048, "seed": SEED},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": n_cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = _parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,98 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py
+times: quantizers bit-exact on sampled rows / 128-row bands, GEMMs within
+tolerance on sampled output rows.
+
+Workloads (fp8_block_scaled_13_b200/inputs.py): attention projections
+(M=8192, QKV 2048->3072, O 2048->2048), SwiGLU gate+up (M=16384,
+2048->12288, 8 channels x50), MLP down-projection with heavy tails
+(M=16384, 6144->2048, Student-t(3) activations, Laplace gradients, zero
+groups), and the full hidden-2048/FFN-6144 block at a ragged M=8000.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_gemm_close, np_u8
+
+pytestmark = pytest.mark.gpu
+
+N_ROWS = 24  # sampled output rows per GEMM
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    import fp8_block_scaled_13_b200 as m
+    from fp8_block_scaled_13_b200 import build
+    build.build()
+    return m
+
+
+def _workload(name):
+    from fp8_block_scaled_13_b200 import inputs
+    if name == "full_block_m8000":
+        return inputs.full_block(seed=4, m=8000)
+    return inputs.WORKLOADS[name]()
+
+
+def _sample(total, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = rng.choice(total, size=min(n, total), replace=False)
+    rows[-1] = total - 1  # always include the last (possibly ragged) row
+    return np.unique(rows).astype(np.int64)
+
+
+def _check_layer(fp8, oracle_mod, L, seed):
+    dev = torch.device("cuda")
+    x, w, dy = L.x.to(dev), L.w.to(dev), L.dy.to(dev)
+    y, xq, wq = fp8.linear_forward(x, w)
+    dyq = fp8.quant_act(dy, "both")
+    dx = fp8.gemm_dgrad(dyq, wq)
+    dw = fp8.gemm_wgrad(dyq, xq)
+    torch.cuda.synchronize()
+    assert fp8.device_status() == 0
+    m, n, k = L.m, L.n, L.k
+
+    # ---- quantizers: weight in full, activations on sampled rows / bands
+    oq, os_ = oracle_mod.quant_weight(L.w)
+    assert np.array_equal(np_u8(wq.s), os_) and np.array_equal(np_u8(wq.q), oq)
+    assert np.array_equal(np_u8(wq.qt), oq.T)
+    rows = _sample(m, 64, seed)
+    for src, q in ((L.x, xq), (L.dy, dyq)):
+        oq, os_ = oracle_mod.quant_rowwise(src[rows])
+        assert np.array_equal(np_u8(q.q)[rows], oq)
+        assert np.array_equal(np_u8(q.s)[:, rows].T, os_)
+        nb = (m + 127) // 128
+        for b in sorted({0, nb - 1, int(seed) % nb}):
+            r0, r1 = b * 128, min(m, b * 128 + 128)
+            oqt, ost = oracle_mod.quant_colwise(src[r0:r1])
+            assert np.array_equal(np_u8(q.qt)[:, r0:r1], oqt)
+            assert np.array_equal(np_u8(q.st)[b, :src.shape[1]], ost[:, 0])
+
+    # ---- GEMMs on sampled output rows
+    rows = _sample(m, N_ROWS, seed + 1)
+    ref = oracle_mod.linear_fprop(L.x[rows], L.w)
+    assert_gemm_close(y[rows.tolist()], ref, oracle_mod, "%s fprop" % L.name)
+    ref = oracle_mod.linear_dgrad(L.dy[rows], L.w)
+    assert_gemm_close(dx[rows.tolist()], ref, oracle_mod, "%s dgrad" % L.name)
+    cols = _sample(n, N_ROWS, seed + 2)
+    ref = oracle_mod.linear_wgrad(L.dy[:, cols].contiguous(), L.x)
+    assert_gemm_close(dw[cols.tolist()], ref, oracle_mod, "%s wgrad" % L.name)
+
+
+@pytest.mark.parametrize("name", ["single_fprop"])
+def test_single_fprop_full(fp8, oracle_mod, name):
+    L = _workload(name).layers[0]
+    y, xq, wq = fp8.linear_forward(L.x.cuda(), L.w.cuda())
+    torch.cuda.synchronize()
+    assert_gemm_close(y, oracle_mod.linear_fprop(L.x, L.w), oracle_mod, "single fprop")
+    q, s = oracle_mod.quant_rowwise(L.x)
+    assert np.array_equal(np_u8(xq.q), q) and np.array_equal(np_u8(xq.s)[:, :L.m].T, s)
+
+
+@pytest.mark.parametrize("name", ["attn_proj", "swiglu_gate_up", "mlp_down_heavy",
+                                  "full_block_m8000"])
+def test_workload_sampled(fp8, oracle_mod, name):
+    wl = _workload(name)
+    for i, L in enumerate(wl.layers):
+        _check_layer(fp8, oracle_mod, L, seed=17 * i + len(name))
+        torch.cuda.empty_cache()

@@ -26,6 +26,7 @@ PURO_COLWISE = 2
 PURO_BOTH = 3
 
 EXPORTS = (
+    "puro_fp8_blocked_scale_bytes",
     "puro_fp8_quant_act",
     "puro_fp8_quant_weight",
     "puro_fp8_gemm_fprop",
@@ -56,17 +57,19 @@ def load() -> ctypes.CDLL:
             "`python -c 'import __graft_entry__ as g; g.build()'`" % LIB_PATH)
     lib = ctypes.CDLL(LIB_PATH)
     P, I, INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
-    lib.puro_fp8_quant_act.argtypes = [P, I, I, I, INT, P, I, P, I, P, I, P, I, P]
-    lib.puro_fp8_quant_weight.argtypes = [P, I, I, I, P, I, P, P, I, P]
-    lib.puro_fp8_gemm_fprop.argtypes = [P, I, P, I, P, I, P, P, I, I, I, I, P]
-    lib.puro_fp8_gemm_dgrad.argtypes = [P, I, P, I, P, I, P, P, I, I, I, I, P]
-    lib.puro_fp8_gemm_wgrad.argtypes = [P, I, P, I, P, I, P, I, P, I, I, I, I, P]
+    lib.puro_fp8_blocked_scale_bytes.argtypes = [I, I]
+    lib.puro_fp8_blocked_scale_bytes.restype = I
+    lib.puro_fp8_quant_act.argtypes = [P, I, I, I, INT, P, I, P, P, I, P, P]
+    lib.puro_fp8_quant_weight.argtypes = [P, I, I, I, P, I, P, P, I, P, P, P]
+    lib.puro_fp8_gemm_fprop.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
+    lib.puro_fp8_gemm_dgrad.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
+    lib.puro_fp8_gemm_wgrad.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
     lib.puro_fp8_device_status.argtypes = [P]
     lib.puro_fp8_status_string.argtypes = [INT]
     lib.puro_fp8_status_string.restype = ctypes.c_char_p
     lib.puro_fp8_test_bounded_wait.argtypes = [I, P]
     for name in EXPORTS:
-        if name != "puro_fp8_status_string":
+        if name not in ("puro_fp8_status_string", "puro_fp8_blocked_scale_bytes"):
             getattr(lib, name).restype = INT
     _lib = lib
     return lib
@@ -76,31 +79,31 @@ def status_string(status: int) -> str:
     return load().puro_fp8_status_string(int(status)).decode()
 
 
-def puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, ld_s, qt, ld_qt, st, ld_st,
-                       stream) -> int:
-    return load().puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, ld_s, qt, ld_qt,
-                                     st, ld_st, stream)
+def puro_fp8_blocked_scale_bytes(rows, groups) -> int:
+    return load().puro_fp8_blocked_scale_bytes(rows, groups)
 
 
-def puro_fp8_quant_weight(w, n, k, ld_w, q, ld_q, s, qt, ld_qt, stream) -> int:
-    return load().puro_fp8_quant_weight(w, n, k, ld_w, q, ld_q, s, qt, ld_qt, stream)
+def puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, qt, ld_qt, st, stream) -> int:
+    return load().puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, qt, ld_qt, st,
+                                     stream)
 
 
-def puro_fp8_gemm_fprop(qx, ld_qx, sx, ld_sx, qw, ld_qw, sw, y, ld_y, m, n, k, stream) -> int:
-    return load().puro_fp8_gemm_fprop(qx, ld_qx, sx, ld_sx, qw, ld_qw, sw, y, ld_y, m, n, k,
+def puro_fp8_quant_weight(w, n, k, ld_w, q, ld_q, s, qt, ld_qt, s_fwd, s_bwd, stream) -> int:
+    return load().puro_fp8_quant_weight(w, n, k, ld_w, q, ld_q, s, qt, ld_qt, s_fwd, s_bwd, stream)
+
+
+def puro_fp8_gemm_fprop(qx, ld_qx, sx, qw, ld_qw, sw_fwd, y, ld_y, m, n, k, stream) -> int:
+    return load().puro_fp8_gemm_fprop(qx, ld_qx, sx, qw, ld_qw, sw_fwd, y, ld_y, m, n, k, stream)
+
+
+def puro_fp8_gemm_dgrad(qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, n, k, stream) -> int:
+    return load().puro_fp8_gemm_dgrad(qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, n, k,
                                       stream)
 
 
-def puro_fp8_gemm_dgrad(qdy, ld_qdy, sdy, ld_sdy, qwt, ld_qwt, sw, dx, ld_dx, m, n, k,
-                        stream) -> int:
-    return load().puro_fp8_gemm_dgrad(qdy, ld_qdy, sdy, ld_sdy, qwt, ld_qwt, sw, dx, ld_dx, m, n,
-                                      k, stream)
-
-
-def puro_fp8_gemm_wgrad(qdyt, ld_qdyt, sdyt, ld_sdyt, qxt, ld_qxt, sxt, ld_sxt, dw, ld_dw, m, n,
-                        k, stream) -> int:
-    return load().puro_fp8_gemm_wgrad(qdyt, ld_qdyt, sdyt, ld_sdyt, qxt, ld_qxt, sxt, ld_sxt, dw,
-                                      ld_dw, m, n, k, stream)
+def puro_fp8_gemm_wgrad(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k, stream) -> int:
+    return load().puro_fp8_gemm_wgrad(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k,
+                                      stream)
 
 
 def puro_fp8_device_status(stream) -> int:

@@ -11,24 +11,36 @@
 //
 // The pages' "Blackwell MXFP8 path" maps onto tcgen05.mma kind::mxf8f6f4 with
 // block scaling: the MMA multiplies each 32-element K slice by one UE8M0 scale
-// per row of A and per row of B.  A 128-group scale is the same for its four
-// 32-element slices, so every slice of a 128-deep K block uses the same scale
-// byte (it is replicated into all four bytes of its TMEM word).
+// per row of A and per row of B, read from TMEM.  A 128-group scale holds for
+// all four 32-element slices of its K block.  The scale arrays come in the
+// blocked layout (include/puro_fp8.h): one 512-byte chunk holds the scales of
+// 128 rows x 4 K blocks exactly as tcgen05.cp expects them in shared memory
+// (16-byte row i = the words of rows i, i+32, i+64, i+96; byte g of a word =
+// K block g), so a chunk goes from global memory to shared memory with one
+// TMA copy and to TMEM with one tcgen05.cp, once per four K blocks; each MMA
+// then selects its byte with the scale-factor id of the instruction
+// descriptor.
 //
-// CTA organisation (one CTA per SM, persistent over output tiles of
-// 128 x BN):
-//   warp 0   : TMA producer -- per 128-deep K block loads the A tile
-//              (128 x 128 B), the B tile (BN x 128 B), the 128 A scales and,
-//              for per-row B scales, the BN B scales into a STAGES-deep ring.
-//              For 128x128-block B scales it stages the tile's scale panel.
-//   warp 1   : MMA issuer and TMEM owner -- rearranges the stage's scales into
-//              the 32-lane x 4-column TMEM scale layout (tcgen05.cp source),
-//              copies them to TMEM, issues four K=32 block-scaled MMAs and
-//              releases the stage with tcgen05.commit.
-//   warps 2-5: epilogue -- tcgen05.ld of the FP32 accumulator (warp w reads
-//              TMEM lanes 32*(w%4)..+31, i.e. tile rows), BF16 conversion,
-//              16-byte stores; masks rows >= rows_a and columns >= rows_b.
-// With NACC = 2 the epilogue of one tile overlaps the MMAs of the next.
+// Tiles are (128*CG) x BN.  With CG = 2 a cluster of two CTAs on two SMs
+// computes one tile with cta_group::2 MMAs: each CTA holds 128 rows of A and
+// BN/2 rows of B in its shared memory (so each SM loads half of B), the
+// leader CTA issues the MMAs for both, and each CTA's TMEM holds its 128 rows
+// of the accumulator.  Scales: each CTA loads the A scales of its own rows
+// and the B scales of all BN rows.  There is no TMA multicast; every CTA
+// loads its own tiles.
+//
+// Warp roles (per CTA, persistent over the tiles of its cluster):
+//   warp 0    : TMA producer -- A, B and (every 4th K block) scale chunks into
+//               a STAGES-deep ring; both CTAs' copies complete on the leader's
+//               full barrier.
+//   warp 1    : TMEM owner; in the leader, MMA issuer -- tcgen05.cp of the
+//               scale chunks, four K=32 MMAs per K block, tcgen05.commit to
+//               release the stage in both CTAs and to publish the tile.
+//   warps 2-9 : epilogue -- warp w reads TMEM lanes 32*(w%4)..+31 (tile rows)
+//               and one half of the columns, releases the accumulator as soon
+//               as its loads completed, then converts to BF16 and stores.
+// With NACC = 2 (BN <= 128) the MMAs of the next tile also overlap the whole
+// epilogue.
 //
 // Every wait is bounded (common.cuh): on expiry the kernel records
 // PURO_ERR_DEVICE_TIMEOUT, stops issuing work, lets its own copies and MMAs
@@ -40,55 +52,63 @@
 namespace puro {
 
 struct GemmParams {
-  int32_t rows_a;   // output rows (M of the tile grid)
+  int32_t rows_a;   // output rows
   int32_t rows_b;   // output cols
   int32_t kblocks;  // ceil(K / 128)
   int32_t tiles_m, tiles_n;
-  // 128x128-block scales of B: scale(j, kb) = bsf[(j/128) * bsf_row + kb * bsf_col]
-  const uint8_t* bsf;
-  int32_t bsf_row, bsf_col;
   __nv_bfloat16* d;  // BF16 [rows_a, rows_b], row stride ldd
   int64_t ldd;
 };
 
-template <int BN>
+template <int CG, int BN>
 struct GemmCfg {
-  static constexpr int kStages = (BN == 256) ? 4 : 5;
-  static constexpr int kNacc = (BN <= 224) ? 2 : 1;
-  static constexpr int kAccStride = 256;          // TMEM columns between accumulators
-  static constexpr int kSfaCol = 480;             // TMEM columns of the A scales (4)
-  static constexpr int kSfbCol = 484;             // TMEM columns of the B scales (8)
-  static constexpr int kNB = (BN + 127) / 128;    // 128-row blocks of B per tile
-  static constexpr int kPanel = kNB * 256;        // block-scale panel bytes (K <= 32768)
-  static constexpr int kPanels = kStages + 1;
+  static_assert(CG == 1 || CG == 2, "CTA group of 1 or 2");
+  static_assert(BN == 128 || BN == 256, "tile width 128 or 256");
+  static constexpr int kBM = 128 * CG;            // tile rows
+  static constexpr int kBNC = BN / CG;            // rows of B in each CTA
+  static constexpr int kNB = BN / 128;            // 128-row scale chunks of B
   static constexpr uint32_t kABytes = 128 * 128;
-  static constexpr uint32_t kBBytes = BN * 128;
+  static constexpr uint32_t kBBytes = kBNC * 128;
+  static constexpr uint32_t kSfaBytes = 512;
+  static constexpr uint32_t kSfbBytes = 512 * kNB;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kStages0 = (int)((222 * 1024) / kStageBytes);
+  static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
+  static constexpr int kNacc = (BN <= 128) ? 2 : 1;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kEpiCols = BN / 2;         // columns per epilogue warp
+  static constexpr int kSfCol = 256;              // TMEM: 2 slots of 16 columns
   // shared memory carve-up (offsets from a 1024-aligned base)
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
-  static constexpr uint32_t kOffSfaRaw = kOffB + kStages * kBBytes;
-  static constexpr uint32_t kOffSfbRaw = kOffSfaRaw + kStages * 128;
-  static constexpr uint32_t kOffSfaIl = kOffSfbRaw + kStages * (kNB * 128);
-  static constexpr uint32_t kOffSfbIl = kOffSfaIl + kStages * 512;
-  static constexpr uint32_t kOffPanel = kOffSfbIl + kStages * kNB * 512;
-  static constexpr uint32_t kOffBar = (kOffPanel + kPanels * kPanel + 15) & ~15u;
+  static constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
+  static constexpr uint32_t kOffSfb = kOffSfa + kStages * kSfaBytes;
+  static constexpr uint32_t kOffBar = kOffSfb + kStages * kSfbBytes;
   static constexpr uint32_t kNumBars = 2 * kStages + 2 * kNacc + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-  // instruction descriptor: E4M3 x E4M3, UE8M0 scales, K-major A and B,
-  // N = BN, M = 128, scale-factor byte 0 for A and B, dense, K = 32.
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(kStages >= 4 && kStages <= 8, "pipeline depth");
+  // Scale chunks are reused every 4 K blocks per TMEM slot pair; stage buffers
+  // are released by the commit that follows the copy, so any depth works.
+  // instruction descriptor: E4M3 x E4M3 (formats 0), UE8M0 scales (bit 23),
+  // K-major A and B, N = BN (bits 17-22, N >> 3), M = 128*CG (bits 24-28,
+  // M >> 4), dense, K = 32; the scale-factor ids (bits 29-30 for A, 4-5 for
+  // B) are or-ed in per MMA.
   static constexpr uint32_t kIdesc =
-      (0u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (0u << 16) |
-      ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(128 >> 4) << 24);
+      ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(kBM >> 4) << 24);
+  static constexpr uint32_t kTxPerStage = CG * (kABytes + kBBytes);
+  static constexpr uint32_t kTxPerSf = CG * (kSfaBytes + kSfbBytes);
 };
 
-template <int BN, bool B_PER_ROW>
-__global__ void __launch_bounds__(192, 1)
+template <int CG, int BN>
+__global__ void __launch_bounds__(GemmCfg<CG, BN>::kThreads, 1)
     gemm_block_scaled_kernel(const __grid_constant__ CUtensorMap tm_a,
                              const __grid_constant__ CUtensorMap tm_b,
                              const __grid_constant__ CUtensorMap tm_sfa,
                              const __grid_constant__ CUtensorMap tm_sfb, const GemmParams p) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<CG, BN>;
   constexpr int S = C::kStages;
   constexpr int NA = C::kNacc;
   extern __shared__ uint8_t smem_raw[];
@@ -105,6 +125,10 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
+  const int cluster_id = blockIdx.x / CG;
+  const int num_clusters = gridDim.x / CG;
   const int num_tiles = p.tiles_m * p.tiles_n;
 
   if (threadIdx.x == 0) {
@@ -114,7 +138,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < NA; ++a) {
       mbar_init(&accf[a], 1);
-      mbar_init(&acce[a], 4);
+      mbar_init(&acce[a], C::kEpiWarps * CG);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -122,14 +146,14 @@ __global__ void __launch_bounds__(192, 1)
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_sfa);
-    if (B_PER_ROW) prefetch_tmap(&tm_sfb);
+    prefetch_tmap(&tm_sfb);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    tmem_alloc<CG>(tmem_slot, 512);
+    tmem_relinquish<CG>();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_or_block_sync<CG>();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -138,42 +162,34 @@ __global__ void __launch_bounds__(192, 1)
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_phase = 0;
-    int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+    for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-      uint8_t* panel = smem + C::kOffPanel + (it % C::kPanels) * C::kPanel;
+      const int a_row = tm * C::kBM + 128 * (int)rank;
+      const int b_row = tn * BN + C::kBNC * (int)rank;
       for (int kb = 0; kb < p.kblocks; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-        if (!B_PER_ROW && kb == 0) {
-          // scale panel of this tile's B rows: panel[h * kblocks + kb]
-          const int n = C::kNB * p.kblocks;
-          for (int idx = lane; idx < n; idx += 32) {
-            const int h = idx / p.kblocks, k = idx - h * p.kblocks;
-            const int jb = tn * (BN / 128) + h;
-            uint8_t v = 127;
-            if (jb * 128 < p.rows_b) v = __ldg(p.bsf + (int64_t)jb * p.bsf_row + (int64_t)k * p.bsf_col);
-            panel[idx] = v;
-          }
-          __syncwarp();
-        }
         if (lane == 0) {
-          const uint32_t bytes = C::kABytes + C::kBBytes + 128 + (B_PER_ROW ? BN : 0);
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(smem + C::kOffA + stage * C::kABytes, &tm_a, kb * 128, tm * 128, &full[stage]);
-          tma_load_2d(smem + C::kOffB + stage * C::kBBytes, &tm_b, kb * 128, tn * BN, &full[stage]);
-          tma_load_2d(smem + C::kOffSfaRaw + stage * 128, &tm_sfa, tm * 128, kb, &full[stage]);
-          if (B_PER_ROW)
-            tma_load_2d(smem + C::kOffSfbRaw + stage * (C::kNB * 128), &tm_sfb, tn * BN, kb,
-                        &full[stage]);
+          const bool sf = (kb & 3) == 0;
+          if (leader)
+            mbar_arrive_expect_tx(&full[stage], C::kTxPerStage + (sf ? C::kTxPerSf : 0u));
+          const uint32_t bar = leader_addr<CG>(&full[stage]);
+          tma_load_2d<CG>(smem + C::kOffA + stage * C::kABytes, &tm_a, kb * 128, a_row, bar);
+          tma_load_2d<CG>(smem + C::kOffB + stage * C::kBBytes, &tm_b, kb * 128, b_row, bar);
+          if (sf) {
+            tma_load_3d<CG>(smem + C::kOffSfa + stage * C::kSfaBytes, &tm_sfa, 0, kb >> 2,
+                            a_row >> 7, bar);
+            tma_load_3d<CG>(smem + C::kOffSfb + stage * C::kSfbBytes, &tm_sfb, 0, kb >> 2,
+                            (tn * BN) >> 7, bar);
+          }
         }
         issued_mask |= 1u << stage;
         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == S) { stage = 0; phase ^= 1; }
       }
     }
-    // let every load this warp issued land before the block can exit
-    if (lane == 0) {
+    // in the leader, let every load of this cluster land before the block can exit
+    if (lane == 0 && leader) {
       for (int s = 0; s < S; ++s)
         if (issued_mask & (1u << s)) {
           volatile int no_abort = 0;
@@ -182,121 +198,104 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
-    int it = 0;
-    bool ok = true;
-    const uint32_t t_sfa = tmem + C::kSfaCol;
-    const uint32_t t_sfb = tmem + C::kSfbCol;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
-      const int acc = it % NA;
-      const uint32_t acc_phase = (it / NA) & 1;
-      const uint8_t* panel = smem + C::kOffPanel + (it % C::kPanels) * C::kPanel;
-      if (!mbar_wait(&acce[acc], acc_phase ^ 1, abort_flag)) break;
-      tc_fence_after();
-      const uint32_t t_acc = tmem + acc * C::kAccStride;
-      for (int kb = 0; kb < p.kblocks; ++kb) {
-        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-        // scales -> tcgen05.cp source layout: 16-byte row `lane` holds the
-        // words of tile rows lane, lane+32, lane+64, lane+96 (byte replicated)
-        {
-          const uint8_t* raw = smem + C::kOffSfaRaw + stage * 128;
-          uint4 w;
-          w.x = raw[lane] * 0x01010101u;
-          w.y = raw[lane + 32] * 0x01010101u;
-          w.z = raw[lane + 64] * 0x01010101u;
-          w.w = raw[lane + 96] * 0x01010101u;
-          *reinterpret_cast<uint4*>(smem + C::kOffSfaIl + stage * 512 + lane * 16) = w;
-        }
+    if (leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++it) {
+        const int acc = it % NA;
+        const uint32_t acc_phase = (it / NA) & 1;
+        if (!mbar_wait(&acce[acc], acc_phase ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t t_acc = tmem + acc * BN;
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t t_sf = tmem + C::kSfCol + 16 * ((kb >> 2) & 1);
+          if (lane == 0) {
+            if ((kb & 3) == 0) {
+              tc_cp_32x128b_warpx4<CG>(t_sf, desc_dense_rows16(smem_u32(smem + C::kOffSfa + stage * C::kSfaBytes)));
 #pragma unroll
-        for (int h = 0; h < C::kNB; ++h) {
-          uint4 w;
-          if (B_PER_ROW) {
-            const uint8_t* raw = smem + C::kOffSfbRaw + stage * (C::kNB * 128) + h * 128;
-            const int base = h * 128 + lane;
-            w.x = (base < BN ? raw[lane] : 0u) * 0x01010101u;
-            w.y = (base + 32 < BN ? raw[lane + 32] : 0u) * 0x01010101u;
-            w.z = (base + 64 < BN ? raw[lane + 64] : 0u) * 0x01010101u;
-            w.w = (base + 96 < BN ? raw[lane + 96] : 0u) * 0x01010101u;
-          } else {
-            const uint32_t v = panel[h * p.kblocks + kb] * 0x01010101u;
-            w = make_uint4(v, v, v, v);
+              for (int h = 0; h < C::kNB; ++h)
+                tc_cp_32x128b_warpx4<CG>(t_sf + 4 + 4 * h,
+                                         desc_dense_rows16(smem_u32(smem + C::kOffSfb + stage * C::kSfbBytes + 512 * h)));
+            }
+            const uint32_t j = (uint32_t)(kb & 3);
+            const uint32_t idesc = C::kIdesc | (j << 29) | (j << 4);
+            const uint64_t adesc = desc_sw128_kmajor(smem_u32(smem + C::kOffA + stage * C::kABytes));
+            const uint64_t bdesc = desc_sw128_kmajor(smem_u32(smem + C::kOffB + stage * C::kBBytes));
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc_mma_mxf8<CG>(t_acc, adesc + 2 * k, bdesc + 2 * k, idesc, t_sf, t_sf + 4,
+                              (kb | k) != 0 ? 1u : 0u);
+            tc_commit_all<CG>(&empty[stage]);
           }
-          *reinterpret_cast<uint4*>(smem + C::kOffSfbIl + (stage * C::kNB + h) * 512 + lane * 16) = w;
+          __syncwarp();
+          if (++stage == S) { stage = 0; phase ^= 1; }
         }
-        fence_proxy_async_smem();
+        if (!ok) break;
+        if (lane == 0) tc_commit_all<CG>(&accf[acc]);
         __syncwarp();
-        if (lane == 0) {
-          tc_cp_32x128b_warpx4(t_sfa, desc_dense_rows16(smem_u32(smem + C::kOffSfaIl + stage * 512)));
-#pragma unroll
-          for (int h = 0; h < C::kNB; ++h)
-            tc_cp_32x128b_warpx4(t_sfb + 4 * h, desc_dense_rows16(smem_u32(
-                                                     smem + C::kOffSfbIl + (stage * C::kNB + h) * 512)));
-          const uint64_t adesc = desc_sw128_kmajor(smem_u32(smem + C::kOffA + stage * C::kABytes));
-          const uint64_t bdesc = desc_sw128_kmajor(smem_u32(smem + C::kOffB + stage * C::kBBytes));
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_mxf8(t_acc, adesc + 2 * k, bdesc + 2 * k, C::kIdesc, t_sfa, t_sfb,
-                        (kb | k) != 0 ? 1u : 0u);
-          tc_commit(&empty[stage]);
-        }
-        __syncwarp();
-        if (++stage == S) { stage = 0; phase ^= 1; }
       }
-      if (!ok) break;
-      if (lane == 0) tc_commit(&accf[acc]);
+      // wait until every MMA and copy this warp issued has completed
+      if (lane == 0) {
+        tc_commit_local<CG>(drain);
+        volatile int no_abort = 0;
+        mbar_wait(drain, 0, &no_abort, 100000000ull);
+      }
       __syncwarp();
     }
-    // wait until every MMA and copy this warp issued has completed
-    if (lane == 0) {
-      tc_commit(drain);
-      volatile int no_abort = 0;
-      mbar_wait(drain, 0, &no_abort, 100000000ull);
-    }
-    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int sp = warp & 3;  // TMEM sub-partition this warp may access
+    const int sp = warp & 3;                 // TMEM sub-partition this warp may access
+    const int half = (warp - 2) >> 2;        // which half of the columns
     const int row_in_tile = sp * 32 + lane;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++it) {
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
       const int acc = it % NA;
       const uint32_t acc_phase = (it / NA) & 1;
       if (!mbar_wait(&accf[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
-      const int grow = tm * 128 + row_in_tile;
-      const uint32_t t_row = tmem + ((uint32_t)(sp * 32) << 16) + acc * C::kAccStride;
-      __nv_bfloat16* drow = p.d + (int64_t)grow * p.ldd + tn * BN;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, r);
-        tmem_ld_wait();
-        if (grow < p.rows_a && tn * BN + c * 32 < p.rows_b) {
-          uint32_t pk[16];
+      const uint32_t t_base =
+          tmem + ((uint32_t)(sp * 32) << 16) + acc * BN + half * C::kEpiCols;
+      uint32_t r[C::kEpiCols];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * e]),
-                                                     __uint_as_float(r[2 * e + 1]));
-            pk[e] = *reinterpret_cast<uint32_t*>(&h);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(drow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-        }
-      }
+      for (int c = 0; c < C::kEpiCols / 32; ++c)
+        tmem_ld_32x32b_x32(t_base + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[acc]);
+      if (lane == 0) mbar_arrive_leader<CG>(&acce[acc]);
+      const int grow = tm * C::kBM + 128 * (int)rank + row_in_tile;
+      const int gcol = tn * BN + half * C::kEpiCols;
+      if (grow < p.rows_a) {
+        __nv_bfloat16* drow = p.d + (int64_t)grow * p.ldd + gcol;
+#pragma unroll
+        for (int c = 0; c < C::kEpiCols / 32; ++c) {
+          if (gcol + c * 32 < p.rows_b) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[c * 32 + 2 * e]),
+                                                       __uint_as_float(r[c * 32 + 2 * e + 1]));
+              pk[e] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(drow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+      }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_or_block_sync<CG>();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 1) tmem_dealloc<CG>(tmem, 512);
 }
 
 }  // namespace puro

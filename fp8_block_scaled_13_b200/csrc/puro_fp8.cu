@@ -22,6 +22,13 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+#ifndef PURO_GEMM_BN
+#define PURO_GEMM_BN 256
+#endif
+#ifndef PURO_GEMM_CG
+#define PURO_GEMM_CG 2
+#endif
+
 struct DeviceInfo {
   bool checked = false;
   bool supported = false;
@@ -88,6 +95,24 @@ int make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer
   return r == CUDA_SUCCESS ? PURO_OK : PURO_ERR_CUDA;
 }
 
+// Blocked scale array of `rows` rows x `groups` groups seen as a 3-D tensor
+// of 32-bit words {128 words per chunk, ceil(groups/4) chunks, ceil(rows/128)
+// row blocks}; a box of {128, 1, nblk} loads nblk consecutive row blocks of
+// one group quadruple.
+int make_map_scales(CUtensorMap* m, const void* base, int64_t rows, int64_t groups, uint32_t nblk) {
+  const uint64_t g4 = (uint64_t)((groups + 3) / 4), rb = (uint64_t)((rows + 127) / 128);
+  cuuint64_t dims[3] = {128, g4, rb};
+  cuuint64_t strides[2] = {512, g4 * 512};
+  cuuint32_t box[3] = {128, 1, nblk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PURO_OK : PURO_ERR_CUDA;
+}
+
+int64_t g4_of(int64_t groups) { return (groups + 3) / 4; }
+
 int launch_status() {
   return cudaGetLastError() == cudaSuccess ? PURO_OK : PURO_ERR_CUDA;
 }
@@ -104,54 +129,60 @@ int launch_quant(const puro::QuantParams& p, int sms, cudaStream_t stream) {
 // ------------------------------------------------------------------ gemm
 
 struct GemmArgs {
-  const void* a;    int64_t lda;     // E4M3 [rows_a, K]
-  const void* sfa;  int64_t ld_sfa;  // group-major [KB][ld_sfa]
-  const void* b;    int64_t ldb;     // E4M3 [rows_b, K]
-  const void* sfb;  int64_t ld_sfb;  // per-row: group-major [KB][ld_sfb]
-  bool b_per_row;
-  const uint8_t* bsf; int64_t bsf_row, bsf_col;  // per-block scales of B
+  const void* a;    int64_t lda;   // E4M3 [rows_a, K]
+  const void* sfa;                 // blocked, rows_a x ceil(K/128) groups
+  const void* b;    int64_t ldb;   // E4M3 [rows_b, K]
+  const void* sfb;                 // blocked, rows_b x ceil(K/128) groups
   void* d; int64_t ldd;
   int64_t rows_a, rows_b, k;
 };
 
-template <int BN, bool PER_ROW>
+template <int CG, int BN>
 int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
-  using C = puro::GemmCfg<BN>;
+  using C = puro::GemmCfg<CG, BN>;
   CUtensorMap ma, mb, msa, msb;
-  const uint64_t kb = (uint64_t)((g.k + 127) / 128);
+  const int64_t kb = (g.k + 127) / 128;
   int st;
   if ((st = make_map_u8(&ma, g.a, g.k, g.rows_a, g.lda, 128, 128, true)) != PURO_OK) return st;
-  if ((st = make_map_u8(&mb, g.b, g.k, g.rows_b, g.ldb, 128, BN, true)) != PURO_OK) return st;
-  if ((st = make_map_u8(&msa, g.sfa, g.rows_a, kb, g.ld_sfa, 128, 1, false)) != PURO_OK) return st;
-  if (PER_ROW) {
-    if ((st = make_map_u8(&msb, g.sfb, g.rows_b, kb, g.ld_sfb, BN, 1, false)) != PURO_OK) return st;
-  } else {
-    msb = msa;  // unused by the kernel
-  }
-  auto kern = puro::gemm_block_scaled_kernel<BN, PER_ROW>;
-  static bool attr_done[kMaxDevices] = {};
+  if ((st = make_map_u8(&mb, g.b, g.k, g.rows_b, g.ldb, 128, C::kBNC, true)) != PURO_OK) return st;
+  if ((st = make_map_scales(&msa, g.sfa, g.rows_a, kb, 1)) != PURO_OK) return st;
+  if ((st = make_map_scales(&msb, g.sfb, g.rows_b, kb, C::kNB)) != PURO_OK) return st;
+  auto kern = puro::gemm_block_scaled_kernel<CG, BN>;
+  static int max_clusters[kMaxDevices] = {};
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  if (!attr_done[dev_id]) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_clusters[dev_id] == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
       return PURO_ERR_CUDA;
-    attr_done[dev_id] = true;
+    int n = 0;
+    cfg.gridDim = dim3(CG * (dev->sms / CG));
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = dev->sms / CG;
+    max_clusters[dev_id] = n;
   }
   puro::GemmParams p;
   p.rows_a = (int32_t)g.rows_a;
   p.rows_b = (int32_t)g.rows_b;
   p.kblocks = (int32_t)kb;
-  p.tiles_m = (int32_t)((g.rows_a + 127) / 128);
+  p.tiles_m = (int32_t)((g.rows_a + C::kBM - 1) / C::kBM);
   p.tiles_n = (int32_t)((g.rows_b + BN - 1) / BN);
-  p.bsf = g.bsf;
-  p.bsf_row = (int32_t)g.bsf_row;
-  p.bsf_col = (int32_t)g.bsf_col;
   p.d = reinterpret_cast<__nv_bfloat16*>(g.d);
   p.ldd = g.ldd;
   const int tiles = p.tiles_m * p.tiles_n;
-  const int grid = tiles < dev->sms ? tiles : dev->sms;
-  kern<<<grid, 192, C::kSmemBytes, stream>>>(ma, mb, msa, msb, p);
+  const int clusters = tiles < max_clusters[dev_id] ? tiles : max_clusters[dev_id];
+  cfg.gridDim = dim3(CG * clusters);
+  if (cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, p) != cudaSuccess) return PURO_ERR_CUDA;
   return launch_status();
 }
 
@@ -168,8 +199,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
       return PURO_ERR_CUDA;
     return PURO_OK;
   }
-  if (g.b_per_row) return launch_gemm_cfg<256, true>(g, dev, stream);
-  return launch_gemm_cfg<256, false>(g, dev, stream);
+  return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN>(g, dev, stream);
 }
 
 // Shape/alignment checks shared by the three GEMMs.
@@ -201,9 +231,14 @@ const char* puro_fp8_status_string(int status) {
   }
 }
 
+int64_t puro_fp8_blocked_scale_bytes(int64_t rows, int64_t groups) {
+  if (rows <= 0 || groups <= 0) return 0;
+  return ((rows + 127) / 128) * g4_of(groups) * 512;
+}
+
 int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int layout,
-                       void* q, int64_t ld_q, void* s, int64_t ld_s, void* qt, int64_t ld_qt,
-                       void* st, int64_t ld_st, void* stream) {
+                       void* q, int64_t ld_q, void* s, void* qt, int64_t ld_qt, void* st,
+                       void* stream) {
   if (layout != PURO_ROWWISE && layout != PURO_COLWISE && layout != PURO_BOTH)
     return PURO_ERR_LAYOUT;
   if (rows < 0 || cols < 0 || rows >= kMaxDim || cols >= kMaxDim) return PURO_ERR_SHAPE;
@@ -214,11 +249,13 @@ int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, 
   const bool row = layout & PURO_ROWWISE, col = layout & PURO_COLWISE;
   if (row) {
     if ((r = check_mat(q, ld_q, cols, 1)) != PURO_OK) return r;
-    if ((r = check_mat(s, ld_s, rows, 1)) != PURO_OK) return r;
+    if (!s) return PURO_ERR_NULL;
+    if (!aligned16(s)) return PURO_ERR_ALIGN;
   }
   if (col) {
     if ((r = check_mat(qt, ld_qt, (rows + 15) / 16 * 16, 1)) != PURO_OK) return r;
-    if ((r = check_mat(st, ld_st, cols, 1)) != PURO_OK) return r;
+    if (!st) return PURO_ERR_NULL;
+    if (!aligned16(st)) return PURO_ERR_ALIGN;
   }
   DeviceInfo* dev = nullptr;
   if ((r = current_device(&dev)) != PURO_OK) return r;
@@ -230,11 +267,11 @@ int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, 
   p.q = static_cast<uint8_t*>(q);
   p.ld_q = ld_q;
   p.s = static_cast<uint8_t*>(s);
-  p.ld_s = ld_s;
+  p.s_g4 = g4_of(cols / 128);
   p.qt = static_cast<uint8_t*>(qt);
   p.ld_qt = ld_qt;
   p.st = static_cast<uint8_t*>(st);
-  p.ld_st = ld_st;
+  p.st_g4 = g4_of((rows + 127) / 128);
   p.tiles_c = cols / 128;
   p.tiles = p.tiles_c * ((rows + 127) / 128);
   cudaStream_t sm = static_cast<cudaStream_t>(stream);
@@ -244,7 +281,8 @@ int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, 
 }
 
 int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, void* q, int64_t ld_q,
-                          void* s, void* qt, int64_t ld_qt, void* stream) {
+                          void* s, void* qt, int64_t ld_qt, void* s_fwd, void* s_bwd,
+                          void* stream) {
   if (n < 0 || k < 0 || n >= kMaxDim || k >= kMaxDim || n % 128 || k % 128) return PURO_ERR_SHAPE;
   if (n == 0 || k == 0) return PURO_OK;
   int r;
@@ -252,6 +290,7 @@ int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, voi
   if ((r = check_mat(q, ld_q, k, 1)) != PURO_OK) return r;
   if (!s) return PURO_ERR_NULL;
   if (qt && (r = check_mat(qt, ld_qt, n, 1)) != PURO_OK) return r;
+  if ((s_fwd && !aligned16(s_fwd)) || (s_bwd && !aligned16(s_bwd))) return PURO_ERR_ALIGN;
   DeviceInfo* dev = nullptr;
   if ((r = current_device(&dev)) != PURO_OK) return r;
   puro::QuantParams p{};
@@ -264,6 +303,10 @@ int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, voi
   p.qt = static_cast<uint8_t*>(qt);
   p.ld_qt = ld_qt;
   p.sw = static_cast<uint8_t*>(s);
+  p.sw_fwd = static_cast<uint8_t*>(s_fwd);
+  p.fwd_g4 = g4_of(k / 128);
+  p.sw_bwd = static_cast<uint8_t*>(s_bwd);
+  p.bwd_g4 = g4_of(n / 128);
   p.tiles_c = k / 128;
   p.tiles = p.tiles_c * (n / 128);
   cudaStream_t sm = static_cast<cudaStream_t>(stream);
@@ -271,51 +314,45 @@ int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, voi
   return launch_quant<true, false, true>(p, dev->sms, sm);
 }
 
-int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx, int64_t ld_sx,
-                        const void* qw, int64_t ld_qw, const void* sw, void* y, int64_t ld_y,
-                        int64_t m, int64_t n, int64_t k, void* stream) {
+int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx, const void* qw,
+                        int64_t ld_qw, const void* sw_fwd, void* y, int64_t ld_y, int64_t m,
+                        int64_t n, int64_t k, void* stream) {
   if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
   if (n % 128 || k % 128) return PURO_ERR_SHAPE;
-  if (k / 128 > puro::GemmCfg<256>::kPanel / puro::GemmCfg<256>::kNB) return PURO_ERR_SHAPE;
   if (m == 0 || n == 0) return PURO_OK;
   int r;
   if ((r = check_mat(y, ld_y, n, 2)) != PURO_OK) return r;
   if (k > 0) {
     if ((r = check_mat(qx, ld_qx, k, 1)) != PURO_OK) return r;
-    if ((r = check_mat(sx, ld_sx, m, 1)) != PURO_OK) return r;
     if ((r = check_mat(qw, ld_qw, k, 1)) != PURO_OK) return r;
-    if (!sw) return PURO_ERR_NULL;
+    if (!sx || !sw_fwd) return PURO_ERR_NULL;
+    if (!aligned16(sx) || !aligned16(sw_fwd)) return PURO_ERR_ALIGN;
   }
-  GemmArgs g{qx, ld_qx, sx, ld_sx, qw, ld_qw, nullptr, 0, false,
-             static_cast<const uint8_t*>(sw), k / 128, 1, y, ld_y, m, n, k};
+  GemmArgs g{qx, ld_qx, sx, qw, ld_qw, sw_fwd, y, ld_y, m, n, k};
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
-int puro_fp8_gemm_dgrad(const void* qdy, int64_t ld_qdy, const void* sdy, int64_t ld_sdy,
-                        const void* qwt, int64_t ld_qwt, const void* sw, void* dx, int64_t ld_dx,
-                        int64_t m, int64_t n, int64_t k, void* stream) {
+int puro_fp8_gemm_dgrad(const void* qdy, int64_t ld_qdy, const void* sdy, const void* qwt,
+                        int64_t ld_qwt, const void* sw_bwd, void* dx, int64_t ld_dx, int64_t m,
+                        int64_t n, int64_t k, void* stream) {
   if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
   if (n % 128 || k % 128) return PURO_ERR_SHAPE;
-  if (n / 128 > puro::GemmCfg<256>::kPanel / puro::GemmCfg<256>::kNB) return PURO_ERR_SHAPE;
   if (m == 0 || k == 0) return PURO_OK;
   int r;
   if ((r = check_mat(dx, ld_dx, k, 2)) != PURO_OK) return r;
   if (n > 0) {
     if ((r = check_mat(qdy, ld_qdy, n, 1)) != PURO_OK) return r;
-    if ((r = check_mat(sdy, ld_sdy, m, 1)) != PURO_OK) return r;
     if ((r = check_mat(qwt, ld_qwt, n, 1)) != PURO_OK) return r;
-    if (!sw) return PURO_ERR_NULL;
+    if (!sdy || !sw_bwd) return PURO_ERR_NULL;
+    if (!aligned16(sdy) || !aligned16(sw_bwd)) return PURO_ERR_ALIGN;
   }
-  // B = W^T [k, n]; its (row j = k-index, group kb = n-block) scale is
-  // sw[kb * (k/128) + j/128].
-  GemmArgs g{qdy, ld_qdy, sdy, ld_sdy, qwt, ld_qwt, nullptr, 0, false,
-             static_cast<const uint8_t*>(sw), 1, k / 128, dx, ld_dx, m, k, n};
+  GemmArgs g{qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, k, n};
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
-int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* sdyt, int64_t ld_sdyt,
-                        const void* qxt, int64_t ld_qxt, const void* sxt, int64_t ld_sxt, void* dw,
-                        int64_t ld_dw, int64_t m, int64_t n, int64_t k, void* stream) {
+int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* sdyt, const void* qxt,
+                        int64_t ld_qxt, const void* sxt, void* dw, int64_t ld_dw, int64_t m,
+                        int64_t n, int64_t k, void* stream) {
   if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
   if (n % 128 || k % 128) return PURO_ERR_SHAPE;
   if (n == 0 || k == 0) return PURO_OK;
@@ -323,12 +360,11 @@ int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* sdyt, int
   if ((r = check_mat(dw, ld_dw, k, 2)) != PURO_OK) return r;
   if (m > 0) {
     if ((r = check_mat(qdyt, ld_qdyt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
-    if ((r = check_mat(sdyt, ld_sdyt, n, 1)) != PURO_OK) return r;
     if ((r = check_mat(qxt, ld_qxt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
-    if ((r = check_mat(sxt, ld_sxt, k, 1)) != PURO_OK) return r;
+    if (!sdyt || !sxt) return PURO_ERR_NULL;
+    if (!aligned16(sdyt) || !aligned16(sxt)) return PURO_ERR_ALIGN;
   }
-  GemmArgs g{qdyt, ld_qdyt, sdyt, ld_sdyt, qxt, ld_qxt, sxt, ld_sxt, true,
-             nullptr, 0, 0, dw, ld_dw, n, k, m};
+  GemmArgs g{qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, n, k, m};
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 

@@ -37,15 +37,25 @@ struct QuantParams {
   int64_t rows, cols, ld_x;
   uint8_t* q;   // codes, same orientation as x (ROW / BLOCK)
   int64_t ld_q;
-  uint8_t* s;   // ROW: group-major scales [cols/128][ld_s]
-  int64_t ld_s;
+  uint8_t* s;   // ROW: blocked scales, rows x cols/128 groups
+  int64_t s_g4;  // ceil(groups / 4) of s
   uint8_t* qt;  // transposed codes [cols][ld_qt] (COL / BLOCK with transpose)
   int64_t ld_qt;
-  uint8_t* st;  // COL: group-major scales [ceil(rows/128)][ld_st]
-  int64_t ld_st;
-  uint8_t* sw;  // BLOCK: scales [rows/128][cols/128]
+  uint8_t* st;  // COL: blocked scales, cols x ceil(rows/128) groups
+  int64_t st_g4;
+  uint8_t* sw;  // BLOCK: compact scales [rows/128][cols/128]
+  uint8_t* sw_fwd;  // BLOCK: optional blocked, rows x cols/128 groups
+  int64_t fwd_g4;
+  uint8_t* sw_bwd;  // BLOCK: optional blocked, cols x rows/128 groups
+  int64_t bwd_g4;
   int64_t tiles_c, tiles;
 };
+
+// Byte offset of (row r, group g) in a blocked scale array whose rows hold
+// g4 = ceil(groups / 4) chunks of 512 bytes per 128-row block.
+__device__ __forceinline__ int64_t blocked_offset(int64_t r, int64_t g, int64_t g4) {
+  return ((r >> 7) * g4 + (g >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (g & 3);
+}
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   uint4 v;
@@ -237,29 +247,24 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(const QuantParams p) {
       }
     }
 
-    // ---- scales
+    // ---- scales (blocked layout); rows past the end hold zeros, so their
+    // scale byte is 127
     if (ROW && !BLOCK && j == 0) {
-      uint8_t* dst = p.s + (c0 / 128) * p.ld_s + r0 + 8 * i;
-      if (r0 + 8 * i + 7 < p.rows) {
-        uint2 b;
-        b.x = (e_row[0] + 127) | ((e_row[1] + 127) << 8) | ((e_row[2] + 127) << 16) |
-              ((uint32_t)(e_row[3] + 127) << 24);
-        b.y = (e_row[4] + 127) | ((e_row[5] + 127) << 8) | ((e_row[6] + 127) << 16) |
-              ((uint32_t)(e_row[7] + 127) << 24);
-        *reinterpret_cast<uint2*>(dst) = b;
-      } else {
+      const int64_t g = c0 / 128;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          if (r0 + 8 * i + k < p.rows) dst[k] = static_cast<uint8_t>(e_row[k] + 127);
-      }
+      for (int k = 0; k < 8; ++k)
+        p.s[blocked_offset(r0 + 8 * i + k, g, p.s_g4)] = static_cast<uint8_t>(e_row[k] + 127);
     }
     if (COL && !BLOCK && i == 0) {
-      uint2 b;
-      b.x = (e_col[0] + 127) | ((e_col[1] + 127) << 8) | ((e_col[2] + 127) << 16) |
-            ((uint32_t)(e_col[3] + 127) << 24);
-      b.y = (e_col[4] + 127) | ((e_col[5] + 127) << 8) | ((e_col[6] + 127) << 16) |
-            ((uint32_t)(e_col[7] + 127) << 24);
-      *reinterpret_cast<uint2*>(p.st + (r0 / 128) * p.ld_st + c0 + 8 * j) = b;
+      const int64_t g = r0 / 128;
+#pragma unroll
+      for (int l = 0; l < 8; ++l)
+        p.st[blocked_offset(c0 + 8 * j + l, g, p.st_g4)] = static_cast<uint8_t>(e_col[l] + 127);
+    }
+    if (BLOCK && tid < 128) {
+      const uint8_t b = static_cast<uint8_t>(e_row[0] + 127);
+      if (p.sw_fwd) p.sw_fwd[blocked_offset(r0 + tid, c0 / 128, p.fwd_g4)] = b;
+      if (p.sw_bwd) p.sw_bwd[blocked_offset(c0 + tid, r0 / 128, p.bwd_g4)] = b;
     }
     if (COL || BLOCK) __syncthreads();  // shared tiles are reused by the next tile
   }

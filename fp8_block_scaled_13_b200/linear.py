@@ -5,8 +5,9 @@ happens here; every step runs in libpuro_fp8.so.
 Layouts (see include/puro_fp8.h):
   * FP8 codes are torch.uint8 tensors (view them as torch.float8_e4m3fn to
     decode); UE8M0 scales are torch.uint8 bytes, scale = 2^(b - 127).
-  * Activation/gradient scales are group-major [groups, ld] with
-    ld = rows rounded up to 16; the valid part is [:, :rows].
+  * Scales a GEMM reads are 1-D uint8 tensors in the blocked layout
+    (512-byte chunks of 128 rows x 4 groups; the index formula is in
+    include/puro_fp8.h).
   * Transposed (COLWISE) codes are [cols, ld] with ld = rows rounded up to 16.
 """
 from __future__ import annotations
@@ -20,6 +21,14 @@ from . import _lib
 
 def _round16(n: int) -> int:
     return (n + 15) // 16 * 16
+
+
+def blocked_scale_bytes(rows: int, groups: int) -> int:
+    return _lib.puro_fp8_blocked_scale_bytes(rows, groups)
+
+
+def _blocked(rows: int, groups: int, dev) -> torch.Tensor:
+    return torch.empty(max(blocked_scale_bytes(rows, groups), 16), dtype=torch.uint8, device=dev)
 
 
 def _stream() -> int:
@@ -46,9 +55,9 @@ class QuantAct:
     rows: int
     cols: int
     q: torch.Tensor | None = None    # [rows, cols] u8
-    s: torch.Tensor | None = None    # [cols/128, ld_s] u8, group-major
+    s: torch.Tensor | None = None    # blocked: rows x cols/128 groups
     qt: torch.Tensor | None = None   # [cols, ld_qt] u8, transposed codes
-    st: torch.Tensor | None = None   # [ceil(rows/128), ld_st] u8, group-major
+    st: torch.Tensor | None = None   # blocked: cols x ceil(rows/128) groups
 
 
 @dataclass
@@ -56,8 +65,10 @@ class QuantWeight:
     n: int
     k: int
     q: torch.Tensor                  # [n, k] u8
-    s: torch.Tensor                  # [n/128, k/128] u8
+    s: torch.Tensor                  # [n/128, k/128] u8, compact
     qt: torch.Tensor | None = None   # [k, n] u8
+    s_fwd: torch.Tensor | None = None  # blocked: n rows x k/128 groups (fprop B scales)
+    s_bwd: torch.Tensor | None = None  # blocked: k rows x n/128 groups (dgrad B scales)
 
 
 def quant_act(x: torch.Tensor, layout: str = "both", out: QuantAct | None = None) -> QuantAct:
@@ -70,17 +81,15 @@ def quant_act(x: torch.Tensor, layout: str = "both", out: QuantAct | None = None
         out = QuantAct(rows, cols)
         if flag & _lib.PURO_ROWWISE:
             out.q = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
-            out.s = torch.empty((cols // 128, _round16(rows)), dtype=torch.uint8, device=dev)
+            out.s = _blocked(rows, cols // 128, dev)
         if flag & _lib.PURO_COLWISE:
             out.qt = torch.empty((cols, _round16(rows)), dtype=torch.uint8, device=dev)
-            out.st = torch.empty(((rows + 127) // 128, _round16(cols)), dtype=torch.uint8, device=dev)
-    z = 0
+            out.st = _blocked(cols, (rows + 127) // 128, dev)
+    ptr = lambda t: t.data_ptr() if t is not None else None
     st = _lib.puro_fp8_quant_act(
         x.data_ptr(), rows, cols, x.stride(0), flag,
-        out.q.data_ptr() if out.q is not None else None, out.q.stride(0) if out.q is not None else z,
-        out.s.data_ptr() if out.s is not None else None, out.s.stride(0) if out.s is not None else z,
-        out.qt.data_ptr() if out.qt is not None else None, out.qt.stride(0) if out.qt is not None else z,
-        out.st.data_ptr() if out.st is not None else None, out.st.stride(0) if out.st is not None else z,
+        ptr(out.q), out.q.stride(0) if out.q is not None else 0, ptr(out.s),
+        ptr(out.qt), out.qt.stride(0) if out.qt is not None else 0, ptr(out.st),
         _stream())
     _check(st, "puro_fp8_quant_act")
     return out
@@ -96,11 +105,14 @@ def quant_weight(w: torch.Tensor, transpose: bool = True, out: QuantWeight | Non
             n, k,
             torch.empty((n, k), dtype=torch.uint8, device=dev),
             torch.empty((n // 128, k // 128), dtype=torch.uint8, device=dev),
-            torch.empty((k, n), dtype=torch.uint8, device=dev) if transpose else None)
+            torch.empty((k, n), dtype=torch.uint8, device=dev) if transpose else None,
+            _blocked(n, k // 128, dev),
+            _blocked(k, n // 128, dev) if transpose else None)
+    ptr = lambda t: t.data_ptr() if t is not None else None
     st = _lib.puro_fp8_quant_weight(
         w.data_ptr(), n, k, w.stride(0), out.q.data_ptr(), out.q.stride(0), out.s.data_ptr(),
-        out.qt.data_ptr() if out.qt is not None else None,
-        out.qt.stride(0) if out.qt is not None else 0, _stream())
+        ptr(out.qt), out.qt.stride(0) if out.qt is not None else 0,
+        ptr(out.s_fwd), ptr(out.s_bwd), _stream())
     _check(st, "puro_fp8_quant_weight")
     return out
 
@@ -113,8 +125,8 @@ def gemm_fprop(xq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) -
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=xq.q.device)
     st = _lib.puro_fp8_gemm_fprop(
-        xq.q.data_ptr(), xq.q.stride(0), xq.s.data_ptr(), xq.s.stride(0),
-        wq.q.data_ptr(), wq.q.stride(0), wq.s.data_ptr(),
+        xq.q.data_ptr(), xq.q.stride(0), xq.s.data_ptr(),
+        wq.q.data_ptr(), wq.q.stride(0), wq.s_fwd.data_ptr(),
         out.data_ptr(), out.stride(0), m, n, k, _stream())
     _check(st, "puro_fp8_gemm_fprop")
     return out
@@ -125,13 +137,13 @@ def gemm_dgrad(dyq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) 
     m, n, k = dyq.rows, dyq.cols, wq.k
     if wq.n != n:
         raise ValueError("dY has %d columns, W has %d rows" % (n, wq.n))
-    if wq.qt is None:
+    if wq.qt is None or wq.s_bwd is None:
         raise ValueError("dgrad needs the transposed weight codes (quant_weight(transpose=True))")
     if out is None:
         out = torch.empty((m, k), dtype=torch.bfloat16, device=dyq.q.device)
     st = _lib.puro_fp8_gemm_dgrad(
-        dyq.q.data_ptr(), dyq.q.stride(0), dyq.s.data_ptr(), dyq.s.stride(0),
-        wq.qt.data_ptr(), wq.qt.stride(0), wq.s.data_ptr(),
+        dyq.q.data_ptr(), dyq.q.stride(0), dyq.s.data_ptr(),
+        wq.qt.data_ptr(), wq.qt.stride(0), wq.s_bwd.data_ptr(),
         out.data_ptr(), out.stride(0), m, n, k, _stream())
     _check(st, "puro_fp8_gemm_dgrad")
     return out
@@ -145,8 +157,8 @@ def gemm_wgrad(dyq: QuantAct, xq: QuantAct, out: torch.Tensor | None = None) -> 
     if out is None:
         out = torch.empty((n, k), dtype=torch.bfloat16, device=dyq.qt.device)
     st = _lib.puro_fp8_gemm_wgrad(
-        dyq.qt.data_ptr(), dyq.qt.stride(0), dyq.st.data_ptr(), dyq.st.stride(0),
-        xq.qt.data_ptr(), xq.qt.stride(0), xq.st.data_ptr(), xq.st.stride(0),
+        dyq.qt.data_ptr(), dyq.qt.stride(0), dyq.st.data_ptr(),
+        xq.qt.data_ptr(), xq.qt.stride(0), xq.st.data_ptr(),
         out.data_ptr(), out.stride(0), m, n, k, _stream())
     _check(st, "puro_fp8_gemm_wgrad")
     return out

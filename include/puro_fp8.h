@@ -29,15 +29,22 @@
  *               is the smallest integer with amax <= 448 * 2^e over the group,
  *               clamped to [-127, 127]; an all-zero group has e = 0 (b = 127).
  *               0xFF is never produced.
- *  - Layouts are row-major; every leading dimension (`ld_*`) is in ELEMENTS of
- *    the array it describes (bytes for the FP8 and UE8M0 arrays) and must make
- *    each row start on a 16-byte boundary.  Every pointer must be 16-byte
- *    aligned.
- *  - Activation/gradient scale arrays are stored GROUP-MAJOR: for a quantized
- *    matrix Q [rows, cols] grouped along cols, the scale of (row r, group g)
- *    is s[g * ld_s + r].  This keeps the 128 scales of one GEMM tile
- *    contiguous so the GEMM loads them with one bulk tensor copy.
- *  - Weight scale arrays are compact row-major [n/128, k/128].
+ *  - Matrices are row-major; every leading dimension (`ld_*`) is in ELEMENTS
+ *    of the array it describes (bytes for FP8 arrays) and must make each row
+ *    start on a 16-byte boundary.  Every pointer must be 16-byte aligned.
+ *  - Scale arrays a GEMM reads are stored in the BLOCKED layout that the
+ *    tensor core's block-scaled MMA consumes (the MX scale-factor layout):
+ *    for an operand with `rows` rows and `groups` 128-wide groups along its
+ *    reduction dimension, the scale of (row r, group g) is the byte at
+ *        ((r / 128) * G4 + g / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + g % 4
+ *    with G4 = ceil(groups / 4); the array holds ceil(rows / 128) * G4 * 512
+ *    bytes (puro_fp8_blocked_scale_bytes).  Every 512-byte chunk covers 128
+ *    rows x 4 groups, so a GEMM tile loads its scales as whole chunks.
+ *    Bytes of groups >= `groups` are never written; bytes of rows >= `rows`
+ *    in the last chunk are written as 127 by the activation quantizer.
+ *  - The canonical weight scale array is compact row-major [n/128, k/128];
+ *    the weight quantizer can also write it expanded to one byte per row in
+ *    the blocked layout, once per GEMM that reads the weight.
  */
 #ifndef PURO_FP8_H
 #define PURO_FP8_H
@@ -72,6 +79,10 @@ enum {
     PURO_BOTH = 3      /* both outputs from one read of x                         */
 };
 
+/* Bytes of a blocked scale array for `rows` rows and `groups` groups
+ * (ceil(rows/128) * ceil(groups/4) * 512); 0 if either is <= 0. */
+PURO_API int64_t puro_fp8_blocked_scale_bytes(int64_t rows, int64_t groups);
+
 /*
  * puro_fp8_quant_act -- online 1x128 quantization of an activation or
  * gradient (the "activations and gradients, one scale per 128 elements along
@@ -79,85 +90,88 @@ enum {
  * paper.rainbus.top step (3)).
  *
  * x      : BF16 [rows, cols], row stride ld_x elements (ld_x >= cols).
- * layout : PURO_ROWWISE, PURO_COLWISE or PURO_BOTH.
+ * layout : PURO_ROWWISE, PURO_COLWISE or PURO_BOTH.  cols % 128 == 0.
  *
  * ROWWISE output (the fprop/dgrad operand: the reduction dim is cols):
- *   cols % 128 == 0 is required.
  *   q  : E4M3 [rows, cols], row stride ld_q bytes (ld_q >= cols).
- *   s  : UE8M0 group-major [cols/128][ld_s], ld_s >= rows; scale of group
- *        (r, g) = x[r, 128g .. 128g+127] at s[g*ld_s + r].
+ *   s  : blocked scales, `rows` rows x cols/128 groups; group (r, g) is
+ *        x[r, 128g .. 128g+127].
  * COLWISE output (the wgrad operand: the reduction dim is rows = tokens):
  *   qt : E4M3 [cols, ld_qt], ld_qt >= rows rounded up to 16; qt[c*ld_qt + r]
  *        is the code of x[r, c].  Bytes [rows, round_up(rows,16)) of each row
  *        are written as 0; bytes beyond are not touched.
- *   st : UE8M0 group-major [ceil(rows/128)][ld_st], ld_st >= cols; the scale of
- *        (column c, row group g) -- rows 128g .. min(128g+127, rows-1), the last
- *        group may be short and only its valid rows enter the amax -- is at
- *        st[g*ld_st + c].
+ *   st : blocked scales, `cols` rows x ceil(rows/128) groups; group (c, g) is
+ *        x[128g .. min(128g+127, rows-1), c] -- the last group may be short
+ *        and only its valid rows enter the amax.
  * Unused outputs may be NULL.  rows == 0 or cols == 0 is a no-op.
  * Limits: rows, cols < 2^31.
  */
-PURO_API int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int layout,
-                       void* q, int64_t ld_q, void* s, int64_t ld_s,
-                       void* qt, int64_t ld_qt, void* st, int64_t ld_st,
-                       void* stream);
+PURO_API int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                int layout, void* q, int64_t ld_q, void* s,
+                                void* qt, int64_t ld_qt, void* st, void* stream);
 
 /*
  * puro_fp8_quant_weight -- 128x128 block quantization of a weight
  * (paper.rainbus.top background and step (3): "weights in 128x128 blocks,
  * one online power-of-two scale each").
  *
- * w  : BF16 [n, k], row stride ld_w elements; n % 128 == 0, k % 128 == 0.
- * q  : E4M3 [n, k], row stride ld_q bytes.
- * s  : UE8M0 [n/128, k/128] compact row-major; s[bn*(k/128) + bk].
- * qt : optional (NULL to skip) E4M3 [k, n], row stride ld_qt bytes, the byte
- *      transpose of q.  Because the blocks are square, block (bk, bn) of qt has
- *      the scale s[bn*(k/128) + bk]; no second scale array exists.  This is the
- *      K-contiguous weight operand of dgrad.
+ * w     : BF16 [n, k], row stride ld_w elements; n % 128 == 0, k % 128 == 0.
+ * q     : E4M3 [n, k], row stride ld_q bytes.
+ * s     : UE8M0 [n/128, k/128] compact row-major; s[bn*(k/128) + bk].
+ * qt    : optional (NULL to skip) E4M3 [k, n], row stride ld_qt bytes, the byte
+ *         transpose of q -- the K-contiguous weight operand of dgrad.  The
+ *         blocks are square, so block (bk, bn) of qt has the scale
+ *         s[bn*(k/128) + bk].
+ * s_fwd : optional blocked scales of q as the fprop B operand: n rows x k/128
+ *         groups, row j of group kb holding s[(j/128)*(k/128) + kb].
+ * s_bwd : optional blocked scales of qt as the dgrad B operand: k rows x n/128
+ *         groups, row j of group nb holding s[nb*(k/128) + j/128].
  */
 PURO_API int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w,
-                          void* q, int64_t ld_q, void* s,
-                          void* qt, int64_t ld_qt, void* stream);
+                                   void* q, int64_t ld_q, void* s,
+                                   void* qt, int64_t ld_qt, void* s_fwd, void* s_bwd,
+                                   void* stream);
 
 /*
  * puro_fp8_gemm_fprop -- Y = X W^T (forward GEMM of paperlayer.ai Appendix C).
  *   Y[i,j] = sum_kb 2^(ex[i,kb] + ew[j/128,kb]) * sum_{k in kb} qx[i,k] qw[j,k]
  * accumulated in FP32 on the tensor cores, rounded once to BF16 (RNE).
- * qx : E4M3 [m, k] (ld_qx),  sx : group-major [k/128][ld_sx]  (quant_act ROWWISE of X)
- * qw : E4M3 [n, k] (ld_qw),  sw : [n/128, k/128]              (quant_weight of W)
+ * qx : E4M3 [m, k] (ld_qx),  sx    : blocked, m rows x k/128 groups (quant_act ROWWISE of X)
+ * qw : E4M3 [n, k] (ld_qw),  sw_fwd: blocked, n rows x k/128 groups (quant_weight s_fwd)
  * y  : BF16 [m, n], row stride ld_y elements.
- * k % 128 == 0, n % 128 == 0, k <= 32768; any m >= 0 (rows >= m are neither
- * read nor written).
+ * k % 128 == 0, n % 128 == 0; any m >= 0 (rows >= m are neither read nor written).
  */
-PURO_API int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx, int64_t ld_sx,
-                        const void* qw, int64_t ld_qw, const void* sw,
-                        void* y, int64_t ld_y, int64_t m, int64_t n, int64_t k, void* stream);
+PURO_API int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx,
+                                 const void* qw, int64_t ld_qw, const void* sw_fwd,
+                                 void* y, int64_t ld_y, int64_t m, int64_t n, int64_t k,
+                                 void* stream);
 
 /*
  * puro_fp8_gemm_dgrad -- dX = dY W (data-gradient GEMM, reduction over n).
- * qdy : E4M3 [m, n] (ld_qdy), sdy : group-major [n/128][ld_sdy] (quant_act ROWWISE of dY)
- * qwt : E4M3 [k, n] (ld_qwt)  -- the `qt` output of puro_fp8_quant_weight
- * sw  : [n/128, k/128]        -- the same weight scale array as fprop
+ * qdy : E4M3 [m, n] (ld_qdy), sdy   : blocked, m rows x n/128 groups (quant_act ROWWISE of dY)
+ * qwt : E4M3 [k, n] (ld_qwt), sw_bwd: blocked, k rows x n/128 groups (quant_weight qt, s_bwd)
  * dx  : BF16 [m, k], row stride ld_dx elements.
- * k % 128 == 0, n % 128 == 0, n <= 32768; any m >= 0.
+ * k % 128 == 0, n % 128 == 0; any m >= 0.
  */
-PURO_API int puro_fp8_gemm_dgrad(const void* qdy, int64_t ld_qdy, const void* sdy, int64_t ld_sdy,
-                        const void* qwt, int64_t ld_qwt, const void* sw,
-                        void* dx, int64_t ld_dx, int64_t m, int64_t n, int64_t k, void* stream);
+PURO_API int puro_fp8_gemm_dgrad(const void* qdy, int64_t ld_qdy, const void* sdy,
+                                 const void* qwt, int64_t ld_qwt, const void* sw_bwd,
+                                 void* dx, int64_t ld_dx, int64_t m, int64_t n, int64_t k,
+                                 void* stream);
 
 /*
  * puro_fp8_gemm_wgrad -- dW = dY^T X (weight-gradient GEMM, reduction over the
  * m tokens, both operands quantized along m as ta-paperlens §3.2 prescribes
  * for gradients and activations).
- * qdyt : E4M3 [n, ld_qdyt], sdyt : group-major [ceil(m/128)][ld_sdyt] (COLWISE of dY)
- * qxt  : E4M3 [k, ld_qxt],  sxt  : group-major [ceil(m/128)][ld_sxt]  (COLWISE of X)
+ * qdyt : E4M3 [n, ld_qdyt], sdyt : blocked, n rows x ceil(m/128) groups (COLWISE of dY)
+ * qxt  : E4M3 [k, ld_qxt],  sxt  : blocked, k rows x ceil(m/128) groups (COLWISE of X)
  * dw   : BF16 [n, k], row stride ld_dw elements.
- * n % 128 == 0, k % 128 == 0; any m >= 0 (a short last token group is read with
- * zero padding; m == 0 writes dW = 0).
+ * n % 128 == 0, k % 128 == 0; any m >= 0 (a short last token group is read
+ * with zero padding; m == 0 writes dW = 0).
  */
-PURO_API int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* sdyt, int64_t ld_sdyt,
-                        const void* qxt, int64_t ld_qxt, const void* sxt, int64_t ld_sxt,
-                        void* dw, int64_t ld_dw, int64_t m, int64_t n, int64_t k, void* stream);
+PURO_API int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* sdyt,
+                                 const void* qxt, int64_t ld_qxt, const void* sxt,
+                                 void* dw, int64_t ld_dw, int64_t m, int64_t n, int64_t k,
+                                 void* stream);
 
 /*
  * puro_fp8_device_status -- synchronizes `stream`, then returns and clears the

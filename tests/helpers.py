@@ -9,11 +9,26 @@ def np_u8(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy()
 
 
+def blocked_index(rows: int, groups: int) -> np.ndarray:
+    """[rows, groups] matrix of byte offsets into a blocked scale array
+    (the index formula of include/puro_fp8.h)."""
+    r = np.arange(rows, dtype=np.int64)[:, None]
+    g = np.arange(groups, dtype=np.int64)[None, :]
+    g4 = (groups + 3) // 4
+    return ((r // 128) * g4 + g // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + g % 4
+
+
+def unblock(s, rows: int, groups: int) -> np.ndarray:
+    """Blocked scale array -> [rows, groups] matrix."""
+    s = np_u8(s) if hasattr(s, "cpu") else np.asarray(s)
+    return s.reshape(-1)[blocked_index(rows, groups)]
+
+
 def gpu_rowwise(xq, rows=None):
     """(q [R,C], s [R,G]) in the oracle's orientation from a QuantAct."""
-    R = xq.rows
+    R, C = xq.rows, xq.cols
     q = np_u8(xq.q)
-    s = np_u8(xq.s)[:, :R].T
+    s = unblock(xq.s, R, C // 128)
     if rows is not None:
         q, s = q[rows], s[rows]
     return q, s
@@ -23,7 +38,7 @@ def gpu_colwise(xq):
     """(qt [C,R], st [C,G]) in the oracle's orientation, plus the zero padding."""
     R, C = xq.rows, xq.cols
     qt_full = np_u8(xq.qt)
-    st = np_u8(xq.st)[:, :C].T
+    st = unblock(xq.st, C, (R + 127) // 128)
     pad = qt_full[:, R:(R + 15) // 16 * 16]
     return qt_full[:, :R], st, pad
 

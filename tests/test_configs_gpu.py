@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_gemm_close, np_u8
+from helpers import assert_gemm_close, np_u8, unblock
 
 pytestmark = pytest.mark.gpu
 
@@ -56,17 +56,21 @@ def _check_layer(fp8, oracle_mod, L, seed):
     oq, os_ = oracle_mod.quant_weight(L.w)
     assert np.array_equal(np_u8(wq.s), os_) and np.array_equal(np_u8(wq.q), oq)
     assert np.array_equal(np_u8(wq.qt), oq.T)
+    assert np.array_equal(unblock(wq.s_fwd, n, k // 128), np.repeat(os_, 128, axis=0))
+    assert np.array_equal(unblock(wq.s_bwd, k, n // 128), np.repeat(os_.T, 128, axis=0))
     rows = _sample(m, 64, seed)
     for src, q in ((L.x, xq), (L.dy, dyq)):
+        cols = src.shape[1]
         oq, os_ = oracle_mod.quant_rowwise(src[rows])
         assert np.array_equal(np_u8(q.q)[rows], oq)
-        assert np.array_equal(np_u8(q.s)[:, rows].T, os_)
+        assert np.array_equal(unblock(q.s, m, cols // 128)[rows], os_)
         nb = (m + 127) // 128
+        st_all = unblock(q.st, cols, nb)
         for b in sorted({0, nb - 1, int(seed) % nb}):
             r0, r1 = b * 128, min(m, b * 128 + 128)
             oqt, ost = oracle_mod.quant_colwise(src[r0:r1])
             assert np.array_equal(np_u8(q.qt)[:, r0:r1], oqt)
-            assert np.array_equal(np_u8(q.st)[b, :src.shape[1]], ost[:, 0])
+            assert np.array_equal(st_all[:, b], ost[:, 0])
 
     # ---- GEMMs on sampled output rows
     rows = _sample(m, N_ROWS, seed + 1)
@@ -86,7 +90,7 @@ def test_single_fprop_full(fp8, oracle_mod, name):
     torch.cuda.synchronize()
     assert_gemm_close(y, oracle_mod.linear_fprop(L.x, L.w), oracle_mod, "single fprop")
     q, s = oracle_mod.quant_rowwise(L.x)
-    assert np.array_equal(np_u8(xq.q), q) and np.array_equal(np_u8(xq.s)[:, :L.m].T, s)
+    assert np.array_equal(np_u8(xq.q), q) and np.array_equal(unblock(xq.s, L.m, L.k // 128), s)
 
 
 @pytest.mark.parametrize("name", ["attn_proj", "swiglu_gate_up", "mlp_down_heavy",

@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import gpu_colwise, gpu_rowwise, np_u8
+from helpers import blocked_index, gpu_colwise, gpu_rowwise, np_u8, unblock
 
 pytestmark = pytest.mark.gpu
 
@@ -112,6 +112,11 @@ def test_quant_weight(fp8, oracle_mod, n, k):
     assert np.array_equal(np_u8(wq.s), os_)
     assert np.array_equal(np_u8(wq.q), oq)
     assert np.array_equal(np_u8(wq.qt), oq.T)
+    # expanded per-row copies in the GEMM's blocked layout
+    fwd = unblock(wq.s_fwd, n, k // 128)
+    bwd = unblock(wq.s_bwd, k, n // 128)
+    assert np.array_equal(fwd, np.repeat(os_, 128, axis=0))
+    assert np.array_equal(bwd, np.repeat(os_.T, 128, axis=0))
 
 
 def test_quant_weight_heavy_tails(fp8, oracle_mod):
@@ -120,7 +125,8 @@ def test_quant_weight_heavy_tails(fp8, oracle_mod):
     torch.cuda.synchronize()
     oq, os_ = oracle_mod.quant_weight(w)
     assert np.array_equal(np_u8(wq.s), os_) and np.array_equal(np_u8(wq.q), oq)
-    assert wq.qt is None
+    assert wq.qt is None and wq.s_bwd is None
+    assert np.array_equal(unblock(wq.s_fwd, 256, 3), np.repeat(os_, 128, axis=0))
 
 
 def test_bounded_wait_reports_timeout(fp8):
@@ -135,3 +141,17 @@ def test_bounded_wait_reports_timeout(fp8):
     x = _rand((128, 128), 14).cuda()
     fp8.quant_act(x, "rowwise")
     torch.cuda.synchronize()
+
+
+def test_blocked_layout_padding_rows(fp8):
+    """Rows past the end of the last 128-row block carry the zero-group byte 127."""
+    x = _rand((200, 256), 15).cuda()
+    xq = fp8.quant_act(x, "rowwise")
+    torch.cuda.synchronize()
+    full = unblock(xq.s, 256, 2)
+    assert np.all(full[200:] == 127)
+
+
+def test_blocked_index_is_a_bijection():
+    idx = blocked_index(384, 8)
+    assert np.unique(idx).size == idx.size and idx.max() == 3 * 2 * 512 - 1

@@ -120,9 +120,32 @@ int launch_status() {
 // ------------------------------------------------------------------ quant
 
 template <bool ROW, bool COL, bool BLOCK>
-int launch_quant(const puro::QuantParams& p, int sms, cudaStream_t stream) {
-  const int64_t grid = p.tiles < (int64_t)sms * 8 ? p.tiles : (int64_t)sms * 8;
-  puro::quant_tile_kernel<ROW, COL, BLOCK><<<(unsigned)grid, 256, 0, stream>>>(p);
+int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, int sms,
+                 cudaStream_t stream) {
+  int st = get_encoder();
+  if (st != PURO_OK) return st;
+  // BF16 input as a 2-D tensor of 16-bit elements {cols, rows}, 128 x 128 boxes
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)p.cols, (cuuint64_t)p.rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld_x * 2};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  if (g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(x), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return PURO_ERR_CUDA;
+  auto kern = puro::quant_kernel<ROW, COL, BLOCK>;
+  constexpr uint32_t smem = puro::quant_smem_bytes();
+  static bool attr_done[kMaxDevices] = {};
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  if (!attr_done[dev_id]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return PURO_ERR_CUDA;
+    attr_done[dev_id] = true;
+  }
+  const int64_t grid = p.tiles < 2 * (int64_t)sms ? p.tiles : 2 * (int64_t)sms;
+  kern<<<(unsigned)grid, puro::kQThreads, smem, stream>>>(m, p);
   return launch_status();
 }
 
@@ -244,6 +267,7 @@ int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, 
   if (rows < 0 || cols < 0 || rows >= kMaxDim || cols >= kMaxDim) return PURO_ERR_SHAPE;
   if (cols % 128) return PURO_ERR_SHAPE;
   if (rows == 0 || cols == 0) return PURO_OK;
+  if ((cols / 128) * ((rows + 127) / 128) >= kMaxDim) return PURO_ERR_SHAPE;
   int r;
   if ((r = check_mat(x, ld_x, cols, 2)) != PURO_OK) return r;
   const bool row = layout & PURO_ROWWISE, col = layout & PURO_COLWISE;
@@ -260,10 +284,8 @@ int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, 
   DeviceInfo* dev = nullptr;
   if ((r = current_device(&dev)) != PURO_OK) return r;
   puro::QuantParams p{};
-  p.x = static_cast<const uint16_t*>(x);
   p.rows = rows;
   p.cols = cols;
-  p.ld_x = ld_x;
   p.q = static_cast<uint8_t*>(q);
   p.ld_q = ld_q;
   p.s = static_cast<uint8_t*>(s);
@@ -272,12 +294,12 @@ int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, 
   p.ld_qt = ld_qt;
   p.st = static_cast<uint8_t*>(st);
   p.st_g4 = g4_of((rows + 127) / 128);
-  p.tiles_c = cols / 128;
-  p.tiles = p.tiles_c * ((rows + 127) / 128);
+  p.tiles_c = (int32_t)(cols / 128);
+  p.tiles = (int32_t)(p.tiles_c * ((rows + 127) / 128));
   cudaStream_t sm = static_cast<cudaStream_t>(stream);
-  if (row && col) return launch_quant<true, true, false>(p, dev->sms, sm);
-  if (row) return launch_quant<true, false, false>(p, dev->sms, sm);
-  return launch_quant<false, true, false>(p, dev->sms, sm);
+  if (row && col) return launch_quant<true, true, false>(x, ld_x, p, dev->sms, sm);
+  if (row) return launch_quant<true, false, false>(x, ld_x, p, dev->sms, sm);
+  return launch_quant<false, true, false>(x, ld_x, p, dev->sms, sm);
 }
 
 int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, void* q, int64_t ld_q,
@@ -285,6 +307,7 @@ int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, voi
                           void* stream) {
   if (n < 0 || k < 0 || n >= kMaxDim || k >= kMaxDim || n % 128 || k % 128) return PURO_ERR_SHAPE;
   if (n == 0 || k == 0) return PURO_OK;
+  if ((k / 128) * (n / 128) >= kMaxDim) return PURO_ERR_SHAPE;
   int r;
   if ((r = check_mat(w, ld_w, k, 2)) != PURO_OK) return r;
   if ((r = check_mat(q, ld_q, k, 1)) != PURO_OK) return r;
@@ -294,10 +317,8 @@ int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, voi
   DeviceInfo* dev = nullptr;
   if ((r = current_device(&dev)) != PURO_OK) return r;
   puro::QuantParams p{};
-  p.x = static_cast<const uint16_t*>(w);
   p.rows = n;
   p.cols = k;
-  p.ld_x = ld_w;
   p.q = static_cast<uint8_t*>(q);
   p.ld_q = ld_q;
   p.qt = static_cast<uint8_t*>(qt);
@@ -307,11 +328,11 @@ int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, voi
   p.fwd_g4 = g4_of(k / 128);
   p.sw_bwd = static_cast<uint8_t*>(s_bwd);
   p.bwd_g4 = g4_of(n / 128);
-  p.tiles_c = k / 128;
-  p.tiles = p.tiles_c * (n / 128);
+  p.tiles_c = (int32_t)(k / 128);
+  p.tiles = (int32_t)(p.tiles_c * (n / 128));
   cudaStream_t sm = static_cast<cudaStream_t>(stream);
-  if (qt) return launch_quant<true, true, true>(p, dev->sms, sm);
-  return launch_quant<true, false, true>(p, dev->sms, sm);
+  if (qt) return launch_quant<true, true, true>(w, ld_w, p, dev->sms, sm);
+  return launch_quant<true, false, true>(w, ld_w, p, dev->sms, sm);
 }
 
 int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx, const void* qw,

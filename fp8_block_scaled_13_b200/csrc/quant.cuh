@@ -8,33 +8,39 @@
 // e clamped to [-127, 127], and every element is encoded round-to-nearest-even
 // with saturation.
 //
-// One kernel serves every layout.  A CTA of 256 threads owns a 128x128 tile of
-// the BF16 input; thread (i, j) = (tid/16, tid%16) holds rows 8i..8i+7 and
-// columns 8j..8j+7 in registers (eight 16-byte loads, one per row; a warp
-// instruction reads two full 256-byte tile rows).  From those registers:
+// One persistent kernel serves every layout.  Each CTA (256 threads, two per
+// SM, so two tiles are processed side by side) walks a strided list of
+// 128x128 tiles of the BF16 input; a TMA ring of kQStages 32 KB tile buffers
+// keeps the next tiles in flight while the current one is processed, and a
+// stage is handed back to the TMA as soon as every thread has copied its part
+// into registers.  Thread (i, j) = (tid/16, tid%16) holds rows 8i..8i+7 and
+// columns 8j..8j+7.  From those registers:
 //   ROW   : row amax by a 16-lane shuffle reduction; codes stored in place.
-//   COL   : column amax by a shuffle + shared-memory reduction across the 8
+//   COL   : column amax by a shuffle + shared-memory reduction over the 8
 //           warps; codes transposed through an XOR-swizzled 16 KB shared tile
 //           (conflict-free 8-byte writes, 16-byte reads) and written out as
-//           full 128-byte rows of the transposed matrix.
+//           128-byte rows of the transposed matrix.
 //   BLOCK : one amax over the whole tile (128x128 weight block); codes written
 //           in place and, optionally, transposed.
 // The amax is taken on the integer BF16 magnitude bits (|x| is itself a BF16,
 // and the order of non-negative floats equals the order of their bits), and
 // the scale exponent comes from the exponent/mantissa fields alone: with
 // amax = 1.f * 2^E, e = E - 8 if 1.f <= 1.75 (mantissa bits <= 0x60), else
-// E - 7.  Scaling by 2^-e is an exact FP32 multiply (no flush to zero: this
-// file must not be built with fast-math), followed by one hardware
-// round-to-nearest-even, saturating conversion to E4M3.
+// E - 7.  Scaling by 2^-e is an exact packed FP32 multiply (no flush to zero:
+// this file must not be built with fast-math), followed by one hardware
+// round-to-nearest-even, saturating conversion to E4M3 per value.
 #pragma once
 
 #include "common.cuh"
 
 namespace puro {
 
+constexpr int kQThreads = 256;
+constexpr int kQStages = 2;
+constexpr uint32_t kQTileBytes = 128 * 128 * 2;
+
 struct QuantParams {
-  const uint16_t* x;  // BF16 bits [rows, cols], row stride ld_x
-  int64_t rows, cols, ld_x;
+  int64_t rows, cols;
   uint8_t* q;   // codes, same orientation as x (ROW / BLOCK)
   int64_t ld_q;
   uint8_t* s;   // ROW: blocked scales, rows x cols/128 groups
@@ -48,21 +54,13 @@ struct QuantParams {
   int64_t fwd_g4;
   uint8_t* sw_bwd;  // BLOCK: optional blocked, cols x rows/128 groups
   int64_t bwd_g4;
-  int64_t tiles_c, tiles;
+  int32_t tiles_c, tiles;
 };
 
 // Byte offset of (row r, group g) in a blocked scale array whose rows hold
 // g4 = ceil(groups / 4) chunks of 512 bytes per 128-row block.
 __device__ __forceinline__ int64_t blocked_offset(int64_t r, int64_t g, int64_t g4) {
   return ((r >> 7) * g4 + (g >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (g & 3);
-}
-
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
 }
 
 // Scale exponent from the BF16 bits of a group's amax (sign already cleared).
@@ -74,75 +72,145 @@ __device__ __forceinline__ int scale_exponent_from_bits(uint32_t a) {
   return e < -127 ? -127 : e;
 }
 
-// 2^-e as an FP32 (e in [-127, 120], so the result is a normal number).
-__device__ __forceinline__ float pow2_neg(int e) {
-  return __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+// 2^-e as an FP32 (e in [-127, 120], so the result is a normal number), in
+// both lanes of a float2.
+__device__ __forceinline__ float2 pow2_neg_x2(int e) {
+  const float f = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+  return make_float2(f, f);
 }
 
-// Two FP32 values -> two E4M3 codes (RNE, satfinite); `lo` in the low byte.
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
+// Two FP32 values -> two E4M3 codes (RNE, satfinite); x.x in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float2 x) {
+  uint16_t c;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(x.y), "f"(x.x));
+  return c;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// Four values (pairs a, b) times 2^-e (s2) -> four E4M3 codes in one word,
+// a.x in the low byte.  The packed multiply is exact (a power of two,
+// subnormals kept), then one RNE saturating conversion per value.
+__device__ __forceinline__ uint32_t encode4(float2 a, float2 b, float2 s2) {
+  return cvt_e4m3x2(__fmul2_rn(a, s2)) | (cvt_e4m3x2(__fmul2_rn(b, s2)) << 16);
+}
+
+// The two BF16 of a packed word widened to FP32 (exact).
+__device__ __forceinline__ float2 bf16x2_f32(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
 
 __device__ __forceinline__ uint32_t word(const uint4& v, int idx) {
   return idx == 0 ? v.x : idx == 1 ? v.y : idx == 2 ? v.z : v.w;
 }
 
 // Element l (0..7) of an 8-BF16 row chunk, widened to FP32.
-__device__ __forceinline__ float elem(const uint4& v, int l) {
+__device__ __forceinline__ float elem_f32(const uint4& v, int l) {
   const uint32_t w = word(v, l >> 1);
-  return (l & 1) ? bf16_hi(w) : bf16_lo(w);
+  return __uint_as_float((l & 1) ? (w & 0xFFFF0000u) : (w << 16));
 }
 
-// Eight codes of one 8-element row chunk, all scaled by `inv`.
-__device__ __forceinline__ uint2 encode_row8(const uint4& v, float inv) {
+// Eight codes of one 8-element row chunk, all scaled by s2.
+__device__ __forceinline__ uint2 encode_row8(const uint4& v, float2 s2) {
   uint2 o;
-  o.x = e4m3x2(bf16_lo(v.x) * inv, bf16_hi(v.x) * inv) |
-        (e4m3x2(bf16_lo(v.y) * inv, bf16_hi(v.y) * inv) << 16);
-  o.y = e4m3x2(bf16_lo(v.z) * inv, bf16_hi(v.z) * inv) |
-        (e4m3x2(bf16_lo(v.w) * inv, bf16_hi(v.w) * inv) << 16);
+  o.x = encode4(bf16x2_f32(v.x), bf16x2_f32(v.y), s2);
+  o.y = encode4(bf16x2_f32(v.z), bf16x2_f32(v.w), s2);
   return o;
 }
 
+// Eight codes of column l of the thread's 8x8 block (rows 0..7), scaled by s2.
+__device__ __forceinline__ uint2 encode_col8(const uint4 (&v)[8], int l, float2 s2) {
+  uint2 o;
+  o.x = encode4(make_float2(elem_f32(v[0], l), elem_f32(v[1], l)),
+                make_float2(elem_f32(v[2], l), elem_f32(v[3], l)), s2);
+  o.y = encode4(make_float2(elem_f32(v[4], l), elem_f32(v[5], l)),
+                make_float2(elem_f32(v[6], l), elem_f32(v[7], l)), s2);
+  return o;
+}
+
+// Larger of the two 16-bit halves.
+__device__ __forceinline__ uint32_t hmax(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
+
+__device__ __forceinline__ uint4 lds_v4(const uint8_t* p) {
+  return *reinterpret_cast<const uint4*>(p);
+}
+
 template <bool ROW, bool COL, bool BLOCK>
-__global__ void __launch_bounds__(256) quant_tile_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kQThreads, 2)
+    quant_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantParams p) {
   constexpr uint32_t kMag = 0x7FFF7FFFu;
-  __shared__ uint32_t col_part[8][16][4];
-  __shared__ uint32_t col_final[64];
-  __shared__ uint32_t blk_part[8];
-  __shared__ __align__(16) uint8_t qt_s[COL ? 128 * 128 : 16];
+  constexpr int kWarps = kQThreads / 32;
+  extern __shared__ uint8_t qsmem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;                                    // kQStages x 32 KB
+  uint8_t* qt_s = smem + kQStages * kQTileBytes;            // 16 KB transposed codes
+  uint32_t* col_part = reinterpret_cast<uint32_t*>(qt_s + 128 * 128);  // [8 warps][16][4]
+  uint32_t* col_final = col_part + kWarps * 64;             // [64]
+  uint32_t* blk_part = col_final + 64;                      // [8]
+  uint64_t* full = reinterpret_cast<uint64_t*>(blk_part + kWarps);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kQStages);
 
   const int tid = threadIdx.x;
   const int i = tid >> 4, j = tid & 15, warp = tid >> 5;
+  // tiles t = blockIdx.x + it * gridDim.x, walked as (row tile, col tile)
+  const int32_t tc_step = (int32_t)(gridDim.x % p.tiles_c), tr_step = (int32_t)(gridDim.x / p.tiles_c);
+  const int32_t my_tiles =
+      (int32_t)blockIdx.x < p.tiles ? (p.tiles - (int32_t)blockIdx.x + (int32_t)gridDim.x - 1) / (int32_t)gridDim.x : 0;
 
-  for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x) {
-    const int64_t r0 = (t / p.tiles_c) * 128;
-    const int64_t c0 = (t % p.tiles_c) * 128;
+  if (tid == 0) {
+    for (int s = 0; s < kQStages; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tm_x);
+  }
+  __syncthreads();
+  // producer-side tile cursor (thread 0 only)
+  int32_t ptr_r = (int32_t)blockIdx.x / p.tiles_c, ptr_c = (int32_t)blockIdx.x % p.tiles_c;
+  int32_t p_it = 0;
+  auto issue_next = [&]() {
+    const int s = p_it % kQStages;
+    mbar_arrive_expect_tx(&full[s], kQTileBytes);
+    tma_load_2d<1>(tiles + s * kQTileBytes, &tm_x, ptr_c * 128, ptr_r * 128, smem_u32(&full[s]));
+    ++p_it;
+    ptr_c += tc_step;
+    ptr_r += tr_step;
+    if (ptr_c >= p.tiles_c) { ptr_c -= p.tiles_c; ++ptr_r; }
+  };
+  if (tid == 0)
+    while (p_it < my_tiles && p_it < kQStages) issue_next();
 
+  int32_t tr = (int32_t)blockIdx.x / p.tiles_c, tc = (int32_t)blockIdx.x % p.tiles_c;
+  for (int32_t it = 0; it < my_tiles; ++it) {
+    const int32_t r0 = tr * 128, c0 = tc * 128;
+    const int s = it % kQStages;
+    const bool ok = mbar_wait(&full[s], (uint32_t)((it / kQStages) & 1), abort_flag);
+    // this thread's 8 rows x 8 columns; rows past the end were filled with 0
     uint4 v[8];
+    const uint8_t* tile = tiles + s * kQTileBytes + (8 * i) * 256 + 16 * j;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = ok ? lds_v4(tile + k * 256) : make_uint4(0, 0, 0, 0);
+    // every thread holds its part: stage s is free again (and if any wait gave
+    // up, the whole block stops here together)
+    if (__syncthreads_or(!ok)) break;
+    if (tid == 0 && p_it < my_tiles) issue_next();
+
+    // ---- magnitudes: per-row amax of this thread's 8 columns (two rows per
+    // word) and per-column-pair amax of its 8 rows, from the same masked words
+    uint32_t rowmax[4] = {0u, 0u, 0u, 0u};
+    uint32_t cm[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int64_t r = r0 + 8 * i + k;
-      v[k] = (r < p.rows) ? ld_stream_v4(p.x + r * p.ld_x + c0 + 8 * j) : make_uint4(0, 0, 0, 0);
-    }
-
-    // ---- row amax (reduced over the 16 lanes sharing i), packed two rows per word
-    uint32_t rowmax[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t m2[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint4& a = v[2 * q + h];
-        const uint32_t m = __vmaxu2(__vmaxu2(a.x & kMag, a.y & kMag), __vmaxu2(a.z & kMag, a.w & kMag));
-        m2[h] = max(m & 0xFFFFu, m >> 16);
+      const uint32_t a0 = v[k].x & kMag, a1 = v[k].y & kMag, a2 = v[k].z & kMag,
+                     a3 = v[k].w & kMag;
+      if (ROW || BLOCK) {
+        const uint32_t m = hmax(__vmaxu2(__vmaxu2(a0, a1), __vmaxu2(a2, a3)));
+        rowmax[k >> 1] |= (k & 1) ? (m << 16) : m;
       }
-      rowmax[q] = m2[0] | (m2[1] << 16);
+      if (COL && !BLOCK) {
+        cm[0] = __vmaxu2(cm[0], a0);
+        cm[1] = __vmaxu2(cm[1], a1);
+        cm[2] = __vmaxu2(cm[2], a2);
+        cm[3] = __vmaxu2(cm[3], a3);
+      }
     }
     if (ROW || BLOCK) {
 #pragma unroll
@@ -153,121 +221,108 @@ __global__ void __launch_bounds__(256) quant_tile_kernel(const QuantParams p) {
       }
     }
 
-    int e_row[8];
-    int e_col[8];
+    int e_blk = 0;
     if (BLOCK) {
       // one exponent for the whole 128x128 block
       uint32_t m = __vmaxu2(__vmaxu2(rowmax[0], rowmax[1]), __vmaxu2(rowmax[2], rowmax[3]));
       m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
-      if ((tid & 31) == 0) blk_part[warp] = max(m & 0xFFFFu, m >> 16);
+      if ((tid & 31) == 0) blk_part[warp] = hmax(m);
       __syncthreads();
       uint32_t bm = 0;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) bm = max(bm, blk_part[w]);
-      const int e = scale_exponent_from_bits(bm);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) e_row[k] = e_col[k] = e;
-      if (tid == 0) p.sw[(r0 / 128) * p.tiles_c + c0 / 128] = static_cast<uint8_t>(e + 127);
-    } else {
-      if (ROW) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          e_row[2 * q] = scale_exponent_from_bits(rowmax[q] & 0xFFFFu);
-          e_row[2 * q + 1] = scale_exponent_from_bits(rowmax[q] >> 16);
-        }
-      }
-      if (COL) {
-        uint32_t cm[4];
-#pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-          uint32_t m = 0;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) m = __vmaxu2(m, word(v[k], pp) & kMag);
-          m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
-          cm[pp] = m;
-        }
-        if ((tid & 16) == 0) {
-#pragma unroll
-          for (int pp = 0; pp < 4; ++pp) col_part[warp][j][pp] = cm[pp];
-        }
-        __syncthreads();
-        if (tid < 64) {
-          uint32_t m = 0;
-#pragma unroll
-          for (int w = 0; w < 8; ++w) m = __vmaxu2(m, col_part[w][tid >> 2][tid & 3]);
-          col_final[tid] = m;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-          const uint32_t m = col_final[j * 4 + pp];
-          e_col[2 * pp] = scale_exponent_from_bits(m & 0xFFFFu);
-          e_col[2 * pp + 1] = scale_exponent_from_bits(m >> 16);
-        }
-      }
+      for (int w = 0; w < kWarps; ++w) bm = max(bm, blk_part[w]);
+      e_blk = scale_exponent_from_bits(bm);
+      if (tid == 0) p.sw[tr * p.tiles_c + tc] = static_cast<uint8_t>(e_blk + 127);
     }
 
-    // ---- in-place codes (ROW, BLOCK)
+    // ---- in-place codes (ROW, BLOCK) and the row scale bytes
     if (ROW || BLOCK) {
+      uint8_t* qrow = p.q + (int64_t)(r0 + 8 * i) * p.ld_q + c0 + 8 * j;
+      // rows 8i..8i+7 share one 32-row group, so their scale bytes sit 16 apart
+      uint8_t* srow = BLOCK ? nullptr : p.s + blocked_offset(r0 + 8 * i, tc, p.s_g4);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const int64_t r = r0 + 8 * i + k;
-        const uint2 o = encode_row8(v[k], pow2_neg(e_row[k]));
-        if (r < p.rows) *reinterpret_cast<uint2*>(p.q + r * p.ld_q + c0 + 8 * j) = o;
+        const uint32_t m = (k & 1) ? (rowmax[k >> 1] >> 16) : (rowmax[k >> 1] & 0xFFFFu);
+        const int e = BLOCK ? e_blk : scale_exponent_from_bits(m);
+        const uint2 o = encode_row8(v[k], pow2_neg_x2(e));
+        if (r0 + 8 * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
+        if (!BLOCK && j == 0) srow[16 * k] = static_cast<uint8_t>(e + 127);
       }
     }
 
     // ---- transposed codes (COL, BLOCK with a transposed copy)
     if (COL) {
-      if (BLOCK && p.qt == nullptr) {
-        // nothing to transpose
-      } else {
+      if (!BLOCK) {
 #pragma unroll
-        for (int l = 0; l < 8; ++l) {
-          const float inv = pow2_neg(e_col[l]);
-          uint2 o;
-          o.x = e4m3x2(elem(v[0], l) * inv, elem(v[1], l) * inv) |
-                (e4m3x2(elem(v[2], l) * inv, elem(v[3], l) * inv) << 16);
-          o.y = e4m3x2(elem(v[4], l) * inv, elem(v[5], l) * inv) |
-                (e4m3x2(elem(v[6], l) * inv, elem(v[7], l) * inv) << 16);
-          // row (8j+l) of the transposed tile, 8-byte chunk i, XOR-swizzled by j
-          *reinterpret_cast<uint2*>(qt_s + (8 * j + l) * 128 + ((i ^ j) << 3)) = o;
+        for (int pp = 0; pp < 4; ++pp)
+          cm[pp] = __vmaxu2(cm[pp], __shfl_xor_sync(0xFFFFFFFFu, cm[pp], 16));
+        if ((tid & 16) == 0)
+          *reinterpret_cast<uint4*>(&col_part[(warp * 16 + j) * 4]) = make_uint4(cm[0], cm[1], cm[2], cm[3]);
+        __syncthreads();
+        if (tid < 64) {
+          uint32_t m = 0;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) m = __vmaxu2(m, col_part[(w * 16 + (tid >> 2)) * 4 + (tid & 3)]);
+          col_final[tid] = m;
         }
         __syncthreads();
+      }
+      const uint4 cf = *reinterpret_cast<const uint4*>(&col_final[j * 4]);
+      // columns 8j..8j+7 share one 32-row group of the blocked array: 16 bytes apart
+      uint8_t* scol = (!BLOCK && i == 0) ? p.st + blocked_offset(c0 + 8 * j, tr, p.st_g4) : nullptr;
 #pragma unroll
-        for (int pass = 0; pass < 4; ++pass) {
-          const int idx = pass * 256 + tid;
-          const int c = idx >> 3, part = idx & 7;
-          const int jj = (c >> 3) & 15;
-          const uint4 w = *reinterpret_cast<const uint4*>(qt_s + c * 128 + ((part ^ (jj >> 1)) << 4));
-          const uint4 o = (jj & 1) ? make_uint4(w.z, w.w, w.x, w.y) : w;
-          const int64_t rr = r0 + 16 * part;
-          if (rr < p.rows) *reinterpret_cast<uint4*>(p.qt + (c0 + c) * p.ld_qt + rr) = o;
+      for (int l = 0; l < 8; ++l) {
+        int e;
+        if (BLOCK) {
+          e = e_blk;
+        } else {
+          const uint32_t m = word(cf, l >> 1);
+          e = scale_exponent_from_bits((l & 1) ? (m >> 16) : (m & 0xFFFFu));
+          if (i == 0) scol[16 * l] = static_cast<uint8_t>(e + 127);
         }
+        const uint2 o = encode_col8(v, l, pow2_neg_x2(e));
+        // row (8j+l) of the transposed tile, 8-byte chunk i, XOR-swizzled by j
+        *reinterpret_cast<uint2*>(qt_s + (8 * j + l) * 128 + ((i ^ j) << 3)) = o;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int pass = 0; pass < 4; ++pass) {
+        const int idx = pass * kQThreads + tid;
+        const int c = idx >> 3, part = idx & 7;
+        const int jj = (c >> 3) & 15;
+        const uint4 w = lds_v4(qt_s + c * 128 + ((part ^ (jj >> 1)) << 4));
+        const uint4 o = (jj & 1) ? make_uint4(w.z, w.w, w.x, w.y) : w;
+        const int32_t rr = r0 + 16 * part;
+        if (rr < p.rows) *reinterpret_cast<uint4*>(p.qt + (int64_t)(c0 + c) * p.ld_qt + rr) = o;
       }
     }
 
-    // ---- scales (blocked layout); rows past the end hold zeros, so their
-    // scale byte is 127
-    if (ROW && !BLOCK && j == 0) {
-      const int64_t g = c0 / 128;
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        p.s[blocked_offset(r0 + 8 * i + k, g, p.s_g4)] = static_cast<uint8_t>(e_row[k] + 127);
-    }
-    if (COL && !BLOCK && i == 0) {
-      const int64_t g = r0 / 128;
-#pragma unroll
-      for (int l = 0; l < 8; ++l)
-        p.st[blocked_offset(c0 + 8 * j + l, g, p.st_g4)] = static_cast<uint8_t>(e_col[l] + 127);
-    }
     if (BLOCK && tid < 128) {
-      const uint8_t b = static_cast<uint8_t>(e_row[0] + 127);
-      if (p.sw_fwd) p.sw_fwd[blocked_offset(r0 + tid, c0 / 128, p.fwd_g4)] = b;
-      if (p.sw_bwd) p.sw_bwd[blocked_offset(c0 + tid, r0 / 128, p.bwd_g4)] = b;
+      const uint8_t b = static_cast<uint8_t>(e_blk + 127);
+      if (p.sw_fwd) p.sw_fwd[blocked_offset(r0 + tid, tc, p.fwd_g4)] = b;
+      if (p.sw_bwd) p.sw_bwd[blocked_offset(c0 + tid, tr, p.bwd_g4)] = b;
     }
     if (COL || BLOCK) __syncthreads();  // shared tiles are reused by the next tile
+    tc += tc_step;
+    tr += tr_step;
+    if (tc >= p.tiles_c) { tc -= p.tiles_c; ++tr; }
   }
+  // Copies are only issued for tiles this CTA processes, and each one was
+  // waited for above, unless a wait gave up; then let the outstanding ones
+  // land (bounded) before the block exits.
+  if (tid == 0 && *abort_flag) {
+    for (int s = 0; s < kQStages; ++s) {
+      volatile int no_abort = 0;
+      mbar_wait(&full[s], 0, &no_abort, 100000000ull);
+      mbar_wait(&full[s], 1, &no_abort, 100000000ull);
+    }
+  }
+}
+
+// Shared memory the quantizer needs (plus alignment slack).
+constexpr uint32_t quant_smem_bytes() {
+  return kQStages * kQTileBytes + 128 * 128 + (kQThreads / 32) * 64 * 4 + 64 * 4 +
+         (kQThreads / 32) * 4 + kQStages * 8 + 16 + 1024;
 }
 
 }  // namespace puro

@@ -92,6 +92,20 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- launch order
+
+// Programmatic dependent launch: kernels are launched so that their prologue
+// may overlap the tail of the kernel before them on the stream.  Every kernel
+// calls pdl_wait() before its first access to global memory another kernel may
+// have written, and pdl_trigger() once its own prologue is done.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- clusters
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

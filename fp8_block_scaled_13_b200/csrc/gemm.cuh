@@ -60,20 +60,29 @@ struct GemmParams {
   int64_t ldd;
 };
 
-template <int CG, int BN>
+#ifndef PURO_GEMM_BK
+#define PURO_GEMM_BK 128
+#endif
+
+template <int CG, int BN, int BK>
 struct GemmCfg {
   static_assert(CG == 1 || CG == 2, "CTA group of 1 or 2");
   static_assert(BN == 128 || BN == 256, "tile width 128 or 256");
+  static_assert(BK == 64 || BK == 128, "stage depth 64 or 128");
   static constexpr int kBM = 128 * CG;            // tile rows
   static constexpr int kBNC = BN / CG;            // rows of B in each CTA
   static constexpr int kNB = BN / 128;            // 128-row scale chunks of B
-  static constexpr uint32_t kABytes = 128 * 128;
-  static constexpr uint32_t kBBytes = kBNC * 128;
+  static constexpr int kSub = 128 / BK;           // stages per 128-deep scale group
+  static constexpr int kStagesPerSf = 4 * kSub;   // stages per scale chunk (4 groups)
+  static constexpr uint32_t kABytes = 128 * BK;
+  static constexpr uint32_t kBBytes = kBNC * BK;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr int kSfSlots = 3;              // shared-memory ring of scale chunks
   static constexpr uint32_t kSfaBytes = 512;
   static constexpr uint32_t kSfbBytes = 512 * kNB;
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-  static constexpr int kStages0 = (int)((222 * 1024) / kStageBytes);
-  static constexpr int kStages = kStages0 > 8 ? 8 : kStages0;
+  static constexpr uint32_t kSfSlotBytes = kSfaBytes + kSfbBytes;
+  static constexpr int kStages0 = (int)((221 * 1024 - kSfSlots * kSfSlotBytes) / kStageBytes);
+  static constexpr int kStages = kStages0 > 16 ? 16 : kStages0;
   static constexpr int kNacc = (BN <= 128) ? 2 : 1;
   static constexpr int kEpiWarps = 8;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -82,16 +91,13 @@ struct GemmCfg {
   // shared memory carve-up (offsets from a 1024-aligned base)
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
-  static constexpr uint32_t kOffSfa = kOffB + kStages * kBBytes;
-  static constexpr uint32_t kOffSfb = kOffSfa + kStages * kSfaBytes;
-  static constexpr uint32_t kOffBar = kOffSfb + kStages * kSfbBytes;
-  static constexpr uint32_t kNumBars = 2 * kStages + 2 * kNacc + 1;
+  static constexpr uint32_t kOffSf = kOffB + kStages * kBBytes;
+  static constexpr uint32_t kOffBar = kOffSf + kSfSlots * kSfSlotBytes;
+  static constexpr uint32_t kNumBars = 2 * kStages + kSfSlots + 2 * kNacc + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  static_assert(kStages >= 4 && kStages <= 8, "pipeline depth");
-  // Scale chunks are reused every 4 K blocks per TMEM slot pair; stage buffers
-  // are released by the commit that follows the copy, so any depth works.
+  static_assert(kStages >= 4, "pipeline depth");
   // instruction descriptor: E4M3 x E4M3 (formats 0), UE8M0 scales (bit 23),
   // K-major A and B, N = BN (bits 17-22, N >> 3), M = 128*CG (bits 24-28,
   // M >> 4), dense, K = 32; the scale-factor ids (bits 29-30 for A, 4-5 for
@@ -99,27 +105,39 @@ struct GemmCfg {
   static constexpr uint32_t kIdesc =
       ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(kBM >> 4) << 24);
   static constexpr uint32_t kTxPerStage = CG * (kABytes + kBBytes);
-  static constexpr uint32_t kTxPerSf = CG * (kSfaBytes + kSfbBytes);
+  static constexpr uint32_t kTxPerSf = CG * kSfSlotBytes;
 };
 
-template <int CG, int BN>
-__global__ void __launch_bounds__(GemmCfg<CG, BN>::kThreads, 1)
+// Shared-memory matrix descriptor of a K-major operand tile whose rows are BK
+// bytes: 128-byte swizzle (8-row groups 1024 B apart) for BK = 128, 64-byte
+// swizzle (8-row groups 512 B apart) for BK = 64.
+template <int BK>
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
+  if (BK == 128) return desc_sw128_kmajor(saddr);
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(512u >> 4) << 32) |
+         (1ull << 46) | (4ull << 61);
+}
+
+template <int CG, int BN, int BK>
+__global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     gemm_block_scaled_kernel(const __grid_constant__ CUtensorMap tm_a,
                              const __grid_constant__ CUtensorMap tm_b,
                              const __grid_constant__ CUtensorMap tm_sfa,
                              const __grid_constant__ CUtensorMap tm_sfb, const GemmParams p) {
-  using C = GemmCfg<CG, BN>;
+  using C = GemmCfg<CG, BN, BK>;
   constexpr int S = C::kStages;
   constexpr int NA = C::kNacc;
+  constexpr int R = C::kSfSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
-  uint64_t* accf = bars + 2 * S;
-  uint64_t* acce = bars + 2 * S + NA;
-  uint64_t* drain = bars + 2 * S + 2 * NA;
+  uint64_t* sfe = bars + 2 * S;                 // scale ring slots free again
+  uint64_t* accf = bars + 2 * S + R;
+  uint64_t* acce = bars + 2 * S + R + NA;
+  uint64_t* drain = bars + 2 * S + R + 2 * NA;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -136,6 +154,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN>::kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    for (int r = 0; r < R; ++r) mbar_init(&sfe[r], 1);
     for (int a = 0; a < NA; ++a) {
       mbar_init(&accf[a], 1);
       mbar_init(&acce[a], C::kEpiWarps * CG);
@@ -156,11 +175,15 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN>::kThreads, 1)
   cluster_or_block_sync<CG>();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // operands may come from the kernel just before this one on the stream
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     int stage = 0;
     uint32_t phase = 0;
+    int sfc = 0;  // scale chunks loaded so far (ring position)
     uint32_t issued_mask = 0, issued_phase = 0;
     bool ok = true;
     for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
@@ -169,20 +192,23 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN>::kThreads, 1)
       const int b_row = tn * BN + C::kBNC * (int)rank;
       for (int kb = 0; kb < p.kblocks; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+        const bool sf = (kb % C::kStagesPerSf) == 0;
+        const int slot = sfc % R;
+        if (sf && !mbar_wait(&sfe[slot], ((sfc / R) & 1) ^ 1, abort_flag)) { ok = false; break; }
         if (lane == 0) {
-          const bool sf = (kb & 3) == 0;
           if (leader)
             mbar_arrive_expect_tx(&full[stage], C::kTxPerStage + (sf ? C::kTxPerSf : 0u));
           const uint32_t bar = leader_addr<CG>(&full[stage]);
-          tma_load_2d<CG>(smem + C::kOffA + stage * C::kABytes, &tm_a, kb * 128, a_row, bar);
-          tma_load_2d<CG>(smem + C::kOffB + stage * C::kBBytes, &tm_b, kb * 128, b_row, bar);
+          tma_load_2d<CG>(smem + C::kOffA + stage * C::kABytes, &tm_a, kb * BK, a_row, bar);
+          tma_load_2d<CG>(smem + C::kOffB + stage * C::kBBytes, &tm_b, kb * BK, b_row, bar);
           if (sf) {
-            tma_load_3d<CG>(smem + C::kOffSfa + stage * C::kSfaBytes, &tm_sfa, 0, kb >> 2,
-                            a_row >> 7, bar);
-            tma_load_3d<CG>(smem + C::kOffSfb + stage * C::kSfbBytes, &tm_sfb, 0, kb >> 2,
-                            (tn * BN) >> 7, bar);
+            uint8_t* sfbuf = smem + C::kOffSf + slot * C::kSfSlotBytes;
+            const int chunk = kb / C::kStagesPerSf;
+            tma_load_3d<CG>(sfbuf, &tm_sfa, 0, chunk, a_row >> 7, bar);
+            tma_load_3d<CG>(sfbuf + C::kSfaBytes, &tm_sfb, 0, chunk, (tn * BN) >> 7, bar);
           }
         }
+        if (sf) ++sfc;
         issued_mask |= 1u << stage;
         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == S) { stage = 0; phase ^= 1; }
@@ -203,6 +229,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN>::kThreads, 1)
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
+      int sfc = 0;  // scale chunks copied to TMEM so far
       for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++it) {
         const int acc = it % NA;
         const uint32_t acc_phase = (it / NA) & 1;
@@ -212,21 +239,29 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN>::kThreads, 1)
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t t_sf = tmem + C::kSfCol + 16 * ((kb >> 2) & 1);
-          if (lane == 0) {
-            if ((kb & 3) == 0) {
-              tc_cp_32x128b_warpx4<CG>(t_sf, desc_dense_rows16(smem_u32(smem + C::kOffSfa + stage * C::kSfaBytes)));
+          if ((kb % C::kStagesPerSf) == 0) {
+            // a new chunk of scales (4 groups of 128 along K) -> TMEM slot sfc & 1;
+            // its shared-memory slot is released once the copy has completed
+            if (lane == 0) {
+              const uint32_t t_new = tmem + C::kSfCol + 16 * (sfc & 1);
+              const uint8_t* sfbuf = smem + C::kOffSf + (sfc % R) * C::kSfSlotBytes;
+              tc_cp_32x128b_warpx4<CG>(t_new, desc_dense_rows16(smem_u32(sfbuf)));
 #pragma unroll
               for (int h = 0; h < C::kNB; ++h)
-                tc_cp_32x128b_warpx4<CG>(t_sf + 4 + 4 * h,
-                                         desc_dense_rows16(smem_u32(smem + C::kOffSfb + stage * C::kSfbBytes + 512 * h)));
+                tc_cp_32x128b_warpx4<CG>(t_new + 4 + 4 * h,
+                                         desc_dense_rows16(smem_u32(sfbuf + C::kSfaBytes + 512 * h)));
+              tc_commit_all<CG>(&sfe[sfc % R]);
             }
-            const uint32_t j = (uint32_t)(kb & 3);
+            ++sfc;
+          }
+          if (lane == 0) {
+            const uint32_t t_sf = tmem + C::kSfCol + 16 * ((sfc - 1) & 1);
+            const uint32_t j = (uint32_t)((kb / C::kSub) & 3);  // 128-group within the chunk
             const uint32_t idesc = C::kIdesc | (j << 29) | (j << 4);
-            const uint64_t adesc = desc_sw128_kmajor(smem_u32(smem + C::kOffA + stage * C::kABytes));
-            const uint64_t bdesc = desc_sw128_kmajor(smem_u32(smem + C::kOffB + stage * C::kBBytes));
+            const uint64_t adesc = desc_kmajor<BK>(smem_u32(smem + C::kOffA + stage * C::kABytes));
+            const uint64_t bdesc = desc_kmajor<BK>(smem_u32(smem + C::kOffB + stage * C::kBBytes));
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < BK / 32; ++k)
               tc_mma_mxf8<CG>(t_acc, adesc + 2 * k, bdesc + 2 * k, idesc, t_sf, t_sf + 4,
                               (kb | k) != 0 ? 1u : 0u);
             tc_commit_all<CG>(&empty[stage]);

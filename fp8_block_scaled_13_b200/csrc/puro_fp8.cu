@@ -81,16 +81,16 @@ int get_encoder() {
 }
 
 // 2-D byte tensor [outer, inner] with row stride `ld` bytes; box {box_inner,
-// box_outer}; optional 128-byte swizzle; out-of-range reads return zero.
+// box_outer} stored with the given shared-memory swizzle; out-of-range reads
+// return zero.
 int make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-                uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+                uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {ld};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PURO_OK : PURO_ERR_CUDA;
 }
@@ -145,7 +145,17 @@ int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, int sm
     attr_done[dev_id] = true;
   }
   const int64_t grid = p.tiles < 2 * (int64_t)sms ? p.tiles : 2 * (int64_t)sms;
-  kern<<<(unsigned)grid, puro::kQThreads, smem, stream>>>(m, p);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(puro::kQThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, m, p) != cudaSuccess) return PURO_ERR_CUDA;
   return launch_status();
 }
 
@@ -160,31 +170,34 @@ struct GemmArgs {
   int64_t rows_a, rows_b, k;
 };
 
-template <int CG, int BN>
+template <int CG, int BN, int BK>
 int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
-  using C = puro::GemmCfg<CG, BN>;
+  using C = puro::GemmCfg<CG, BN, BK>;
   CUtensorMap ma, mb, msa, msb;
   const int64_t kb = (g.k + 127) / 128;
   int st;
-  if ((st = make_map_u8(&ma, g.a, g.k, g.rows_a, g.lda, 128, 128, true)) != PURO_OK) return st;
-  if ((st = make_map_u8(&mb, g.b, g.k, g.rows_b, g.ldb, 128, C::kBNC, true)) != PURO_OK) return st;
+  const CUtensorMapSwizzle sw = BK == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if ((st = make_map_u8(&ma, g.a, g.k, g.rows_a, g.lda, BK, 128, sw)) != PURO_OK) return st;
+  if ((st = make_map_u8(&mb, g.b, g.k, g.rows_b, g.ldb, BK, C::kBNC, sw)) != PURO_OK) return st;
   if ((st = make_map_scales(&msa, g.sfa, g.rows_a, kb, 1)) != PURO_OK) return st;
   if ((st = make_map_scales(&msb, g.sfb, g.rows_b, kb, C::kNB)) != PURO_OK) return st;
-  auto kern = puro::gemm_block_scaled_kernel<CG, BN>;
+  auto kern = puro::gemm_block_scaled_kernel<CG, BN, BK>;
   static int max_clusters[kMaxDevices] = {};
   int dev_id = 0;
   cudaGetDevice(&dev_id);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;  // the occupancy query below uses the cluster attribute only
   if (max_clusters[dev_id] == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
@@ -197,7 +210,7 @@ int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
   puro::GemmParams p;
   p.rows_a = (int32_t)g.rows_a;
   p.rows_b = (int32_t)g.rows_b;
-  p.kblocks = (int32_t)kb;
+  p.kblocks = (int32_t)((g.k + BK - 1) / BK);
   p.tiles_m = (int32_t)((g.rows_a + C::kBM - 1) / C::kBM);
   p.tiles_n = (int32_t)((g.rows_b + BN - 1) / BN);
   p.d = reinterpret_cast<__nv_bfloat16*>(g.d);
@@ -205,6 +218,7 @@ int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
   const int tiles = p.tiles_m * p.tiles_n;
   const int clusters = tiles < max_clusters[dev_id] ? tiles : max_clusters[dev_id];
   cfg.gridDim = dim3(CG * clusters);
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, p) != cudaSuccess) return PURO_ERR_CUDA;
   return launch_status();
 }
@@ -222,7 +236,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
       return PURO_ERR_CUDA;
     return PURO_OK;
   }
-  return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN>(g, dev, stream);
+  return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN, PURO_GEMM_BK>(g, dev, stream);
 }
 
 // Shape/alignment checks shared by the three GEMMs.

@@ -163,6 +163,9 @@ __global__ void __launch_bounds__(kQThreads, 2)
     prefetch_tmap(&tm_x);
   }
   __syncthreads();
+  // the input may come from the kernel just before this one on the stream
+  pdl_wait();
+  pdl_trigger();
   // producer-side tile cursor (thread 0 only)
   int32_t ptr_r = (int32_t)blockIdx.x / p.tiles_c, ptr_c = (int32_t)blockIdx.x % p.tiles_c;
   int32_t p_it = 0;

@@ -88,6 +88,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait by every lane of a converged warp, with one verdict for the whole
+// warp (lanes time out on their own clocks; the vote keeps them together so
+// that full-mask warp instructions after the wait see all 32 lanes).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -107,6 +116,23 @@ __device__ __forceinline__ void pdl_trigger() {
 }
 
 // ---------------------------------------------------------------- clusters
+
+// True in exactly one lane of the (converged) warp.  Single-thread work of a
+// warp that otherwise runs converged (issuing tcgen05 MMAs, copies and
+// commits, TMA copies) goes under this instead of a lane-id test: issuing the
+// MMA stream from a lane-id branch was measured to add ~150 cycles per 128-deep
+// K block (four 256x256x32 MMAs) on top of the 512 the tensor pipe needs.
+// With a full member mask the elected lane is the same every time, so commits
+// issued under it track the MMAs issued under it.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

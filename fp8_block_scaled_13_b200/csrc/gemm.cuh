@@ -191,11 +191,11 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       const int a_row = tm * C::kBM + 128 * (int)rank;
       const int b_row = tn * BN + C::kBNC * (int)rank;
       for (int kb = 0; kb < p.kblocks; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
         const bool sf = (kb % C::kStagesPerSf) == 0;
         const int slot = sfc % R;
-        if (sf && !mbar_wait(&sfe[slot], ((sfc / R) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (lane == 0) {
+        if (sf && !mbar_wait_warp(&sfe[slot], ((sfc / R) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (elect_one()) {
           if (leader)
             mbar_arrive_expect_tx(&full[stage], C::kTxPerStage + (sf ? C::kTxPerSf : 0u));
           const uint32_t bar = leader_addr<CG>(&full[stage]);
@@ -230,19 +230,21 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       int it = 0;
       bool ok = true;
       int sfc = 0;  // scale chunks copied to TMEM so far
+      const uint64_t adesc0 = desc_kmajor<BK>(smem_u32(smem + C::kOffA));
+      const uint64_t bdesc0 = desc_kmajor<BK>(smem_u32(smem + C::kOffB));
       for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++it) {
         const int acc = it % NA;
         const uint32_t acc_phase = (it / NA) & 1;
-        if (!mbar_wait(&acce[acc], acc_phase ^ 1, abort_flag)) break;
+        if (!mbar_wait_warp(&acce[acc], acc_phase ^ 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t t_acc = tmem + acc * BN;
         for (int kb = 0; kb < p.kblocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           if ((kb % C::kStagesPerSf) == 0) {
             // a new chunk of scales (4 groups of 128 along K) -> TMEM slot sfc & 1;
             // its shared-memory slot is released once the copy has completed
-            if (lane == 0) {
+            if (elect_one()) {
               const uint32_t t_new = tmem + C::kSfCol + 16 * (sfc & 1);
               const uint8_t* sfbuf = smem + C::kOffSf + (sfc % R) * C::kSfSlotBytes;
               tc_cp_32x128b_warpx4<CG>(t_new, desc_dense_rows16(smem_u32(sfbuf)));
@@ -254,31 +256,28 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
             }
             ++sfc;
           }
-          if (lane == 0) {
+          if (elect_one()) {
             const uint32_t t_sf = tmem + C::kSfCol + 16 * ((sfc - 1) & 1);
             const uint32_t j = (uint32_t)((kb / C::kSub) & 3);  // 128-group within the chunk
             const uint32_t idesc = C::kIdesc | (j << 29) | (j << 4);
-            const uint64_t adesc = desc_kmajor<BK>(smem_u32(smem + C::kOffA + stage * C::kABytes));
-            const uint64_t bdesc = desc_kmajor<BK>(smem_u32(smem + C::kOffB + stage * C::kBBytes));
+            // start-address field (16-byte units) of the stage's descriptors
+            const uint64_t adesc = adesc0 + (uint64_t)(stage * (C::kABytes >> 4));
+            const uint64_t bdesc = bdesc0 + (uint64_t)(stage * (C::kBBytes >> 4));
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k)
               tc_mma_mxf8<CG>(t_acc, adesc + 2 * k, bdesc + 2 * k, idesc, t_sf, t_sf + 4,
                               (kb | k) != 0 ? 1u : 0u);
             tc_commit_all<CG>(&empty[stage]);
           }
-          __syncwarp();
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        if (lane == 0) tc_commit_all<CG>(&accf[acc]);
-        __syncwarp();
+        if (elect_one()) tc_commit_all<CG>(&accf[acc]);
       }
       // wait until every MMA and copy this warp issued has completed
-      if (lane == 0) {
-        tc_commit_local<CG>(drain);
-        volatile int no_abort = 0;
-        mbar_wait(drain, 0, &no_abort, 100000000ull);
-      }
+      if (elect_one()) tc_commit_local<CG>(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort, 100000000ull);
       __syncwarp();
     }
   } else {

@@ -38,9 +38,21 @@
 //               release the stage in both CTAs and to publish the tile.
 //   warps 2-9 : epilogue -- warp w reads TMEM lanes 32*(w%4)..+31 (tile rows)
 //               and one half of the columns, releases the accumulator as soon
-//               as its loads completed, then converts to BF16 and stores.
-// With NACC = 2 (BN <= 128) the MMAs of the next tile also overlap the whole
-// epilogue.
+//               as its loads completed, then converts to BF16 and writes the
+//               rows through shared memory, 32 columns at a time, with TMA
+//               tensor stores (64-byte row segments; one thread per row
+//               storing straight to global memory touched 32 lines per
+//               instruction and was the throughput limit of the kernel).
+//
+// TMEM (512 columns) holds two accumulators, so the MMAs of the next tile
+// overlap the epilogue of the previous one.  With BN = 256 the two 256-column
+// accumulators fill TMEM, and the scale factors of a tile (two 16-column
+// slots) live in the last 32 columns of the OTHER accumulator: the epilogue
+// drains those 32 columns first and hands them over (barrier `sft`), so the
+// next tile can start after a 32-column drain instead of a 256-column one.
+// The next-but-one tile, which accumulates into those columns again, starts
+// only after this tile's MMAs completed (its own `sft` wait follows this
+// tile's accumulator commit), so scales are never overwritten while in use.
 //
 // Every wait is bounded (common.cuh): on expiry the kernel records
 // PURO_ERR_DEVICE_TIMEOUT, stops issuing work, lets its own copies and MMAs
@@ -55,13 +67,14 @@ struct GemmParams {
   int32_t rows_a;   // output rows
   int32_t rows_b;   // output cols
   int32_t kblocks;  // ceil(K / 128)
-  int32_t tiles_m, tiles_n;
-  __nv_bfloat16* d;  // BF16 [rows_a, rows_b], row stride ldd
-  int64_t ldd;
+  int32_t tiles_m, tiles_n;  // the BF16 output goes through the tm_d tensor map
 };
 
 #ifndef PURO_GEMM_BK
 #define PURO_GEMM_BK 128
+#endif
+#ifndef PURO_GEMM_EPI_BUFS
+#define PURO_GEMM_EPI_BUFS 1
 #endif
 
 template <int CG, int BN, int BK>
@@ -81,19 +94,26 @@ struct GemmCfg {
   static constexpr uint32_t kSfaBytes = 512;
   static constexpr uint32_t kSfbBytes = 512 * kNB;
   static constexpr uint32_t kSfSlotBytes = kSfaBytes + kSfbBytes;
-  static constexpr int kStages0 = (int)((221 * 1024 - kSfSlots * kSfSlotBytes) / kStageBytes);
-  static constexpr int kStages = kStages0 > 16 ? 16 : kStages0;
-  static constexpr int kNacc = (BN <= 128) ? 2 : 1;
   static constexpr int kEpiWarps = 8;
+  // epilogue staging: per warp kEpiBufs buffers of 32 rows x 32 BF16 columns
+  static constexpr int kEpiBufs = PURO_GEMM_EPI_BUFS;
+  static constexpr uint32_t kEpiChunkBytes = 32 * 32 * 2;
+  static constexpr uint32_t kEpiBytes = kEpiWarps * kEpiBufs * kEpiChunkBytes;
+  static constexpr int kStages0 =
+      (int)((221 * 1024 - kSfSlots * kSfSlotBytes - kEpiBytes - 1024) / kStageBytes);
+  static constexpr int kStages = kStages0 > 16 ? 16 : kStages0;
+  static constexpr int kNacc = 2;                 // accumulators in TMEM
+  static constexpr bool kSfInTail = (BN == 256);  // scales in the other accumulator's tail
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kEpiCols = BN / 2;         // columns per epilogue warp
-  static constexpr int kSfCol = 256;              // TMEM: 2 slots of 16 columns
+  static constexpr int kSfCol = 256;              // BN = 128: 2 slots of 16 columns after both accumulators
   // shared memory carve-up (offsets from a 1024-aligned base)
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * kABytes;
   static constexpr uint32_t kOffSf = kOffB + kStages * kBBytes;
-  static constexpr uint32_t kOffBar = kOffSf + kSfSlots * kSfSlotBytes;
-  static constexpr uint32_t kNumBars = 2 * kStages + kSfSlots + 2 * kNacc + 1;
+  static constexpr uint32_t kOffEpi = (kOffSf + kSfSlots * kSfSlotBytes + 1023) / 1024 * 1024;
+  static constexpr uint32_t kOffBar = kOffEpi + kEpiBytes;
+  static constexpr uint32_t kNumBars = 2 * kStages + kSfSlots + 3 * kNacc + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -123,7 +143,8 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     gemm_block_scaled_kernel(const __grid_constant__ CUtensorMap tm_a,
                              const __grid_constant__ CUtensorMap tm_b,
                              const __grid_constant__ CUtensorMap tm_sfa,
-                             const __grid_constant__ CUtensorMap tm_sfb, const GemmParams p) {
+                             const __grid_constant__ CUtensorMap tm_sfb,
+                             const __grid_constant__ CUtensorMap tm_d, const GemmParams p) {
   using C = GemmCfg<CG, BN, BK>;
   constexpr int S = C::kStages;
   constexpr int NA = C::kNacc;
@@ -138,6 +159,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
   uint64_t* accf = bars + 2 * S + R;
   uint64_t* acce = bars + 2 * S + R + NA;
   uint64_t* drain = bars + 2 * S + R + 2 * NA;
+  uint64_t* sft = bars + 2 * S + R + 2 * NA + 1;  // accumulator tail (scale area) drained
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -158,6 +180,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     for (int a = 0; a < NA; ++a) {
       mbar_init(&accf[a], 1);
       mbar_init(&acce[a], C::kEpiWarps * CG);
+      mbar_init(&sft[a], (C::kEpiWarps / 2) * CG);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -166,6 +189,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_sfa);
     prefetch_tmap(&tm_sfb);
+    prefetch_tmap(&tm_d);
   }
   if (warp == 1) {
     tmem_alloc<CG>(tmem_slot, 512);
@@ -236,8 +260,14 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
         const int acc = it % NA;
         const uint32_t acc_phase = (it / NA) & 1;
         if (!mbar_wait_warp(&acce[acc], acc_phase ^ 1, abort_flag)) break;
+        // scale slots of this tile: the tail of the other accumulator, free once
+        // the previous tile's epilogue has read it
+        if (C::kSfInTail && it > 0 &&
+            !mbar_wait_warp(&sft[acc ^ 1], ((it - 1) / NA) & 1, abort_flag))
+          break;
         tc_fence_after();
         const uint32_t t_acc = tmem + acc * BN;
+        const uint32_t t_sfreg = tmem + (C::kSfInTail ? (uint32_t)((acc ^ 1) * BN + BN - 32) : C::kSfCol);
         for (int kb = 0; kb < p.kblocks; ++kb) {
           if (!mbar_wait_warp(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -245,7 +275,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
             // a new chunk of scales (4 groups of 128 along K) -> TMEM slot sfc & 1;
             // its shared-memory slot is released once the copy has completed
             if (elect_one()) {
-              const uint32_t t_new = tmem + C::kSfCol + 16 * (sfc & 1);
+              const uint32_t t_new = t_sfreg + 16 * (sfc & 1);
               const uint8_t* sfbuf = smem + C::kOffSf + (sfc % R) * C::kSfSlotBytes;
               tc_cp_32x128b_warpx4<CG>(t_new, desc_dense_rows16(smem_u32(sfbuf)));
 #pragma unroll
@@ -257,7 +287,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
             ++sfc;
           }
           if (elect_one()) {
-            const uint32_t t_sf = tmem + C::kSfCol + 16 * ((sfc - 1) & 1);
+            const uint32_t t_sf = t_sfreg + 16 * ((sfc - 1) & 1);
             const uint32_t j = (uint32_t)((kb / C::kSub) & 3);  // 128-group within the chunk
             const uint32_t idesc = C::kIdesc | (j << 29) | (j << 4);
             // start-address field (16-byte units) of the stage's descriptors
@@ -284,7 +314,8 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int sp = warp & 3;                 // TMEM sub-partition this warp may access
     const int half = (warp - 2) >> 2;        // which half of the columns
-    const int row_in_tile = sp * 32 + lane;
+    uint8_t* ebuf = smem + C::kOffEpi + (warp - 2) * C::kEpiBufs * C::kEpiChunkBytes;
+    int ebufc = 0;  // chunks staged so far (staging buffer ring position)
     int it = 0;
     for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++it) {
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
@@ -295,20 +326,43 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       const uint32_t t_base =
           tmem + ((uint32_t)(sp * 32) << 16) + acc * BN + half * C::kEpiCols;
       uint32_t r[C::kEpiCols];
+      constexpr int NC = C::kEpiCols / 32;
+      if (C::kSfInTail && half == 1) {
+        // the last 32 columns first: the next tile's scales go there
+        tmem_ld_32x32b_x32(t_base + (NC - 1) * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[(NC - 1) * 32]));
+        tmem_ld_wait();
+        regs_after_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[(NC - 1) * 32]));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_leader<CG>(&sft[acc]);
 #pragma unroll
-      for (int c = 0; c < C::kEpiCols / 32; ++c)
-        tmem_ld_32x32b_x32(t_base + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-      tmem_ld_wait();
+        for (int c = 0; c < NC - 1; ++c)
+          tmem_ld_32x32b_x32(t_base + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < NC - 1; ++c) regs_after_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+          tmem_ld_32x32b_x32(t_base + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < NC; ++c) regs_after_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader<CG>(&acce[acc]);
-      const int grow = tm * C::kBM + 128 * (int)rank + row_in_tile;
+      // BF16 rows through this warp's staging buffers: lane = row, 64 bytes
+      // (32 columns) per chunk; one TMA store per chunk writes 32 rows x 64 B
+      const int row0 = tm * C::kBM + 128 * (int)rank + sp * 32;
       const int gcol = tn * BN + half * C::kEpiCols;
-      if (grow < p.rows_a) {
-        __nv_bfloat16* drow = p.d + (int64_t)grow * p.ldd + gcol;
+      if (row0 < p.rows_a) {
 #pragma unroll
-        for (int c = 0; c < C::kEpiCols / 32; ++c) {
+        for (int c = 0; c < NC; ++c) {
           if (gcol + c * 32 < p.rows_b) {
+            uint8_t* buf = ebuf + (ebufc % C::kEpiBufs) * C::kEpiChunkBytes;
+            if (lane == 0) bulk_wait_group_read<C::kEpiBufs - 1>();
+            __syncwarp();
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -316,14 +370,24 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
                                                        __uint_as_float(r[c * 32 + 2 * e + 1]));
               pk[e] = *reinterpret_cast<uint32_t*>(&h);
             }
-            uint4* dst = reinterpret_cast<uint4*>(drow + c * 32);
+            uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_d, buf, gcol + c * 32, row0);
+              bulk_commit_group();
+            }
+            ++ebufc;
           }
         }
       }
     }
+    // the staging buffers must stay valid until the stores have read them
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
   }
 
   tc_fence_before();

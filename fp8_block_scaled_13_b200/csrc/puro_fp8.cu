@@ -181,6 +181,18 @@ int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
   if ((st = make_map_u8(&mb, g.b, g.k, g.rows_b, g.ldb, BK, C::kBNC, sw)) != PURO_OK) return st;
   if ((st = make_map_scales(&msa, g.sfa, g.rows_a, kb, 1)) != PURO_OK) return st;
   if ((st = make_map_scales(&msb, g.sfb, g.rows_b, kb, C::kNB)) != PURO_OK) return st;
+  // BF16 output [rows_a, rows_b], row stride ldd elements; 32 x 32 store boxes
+  CUtensorMap md;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)g.rows_b, (cuuint64_t)g.rows_a};
+    cuuint64_t strides[1] = {(cuuint64_t)g.ldd * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    if (g_encode(&md, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.d, dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return PURO_ERR_CUDA;
+  }
   auto kern = puro::gemm_block_scaled_kernel<CG, BN, BK>;
   static int max_clusters[kMaxDevices] = {};
   int dev_id = 0;
@@ -213,13 +225,11 @@ int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
   p.kblocks = (int32_t)((g.k + BK - 1) / BK);
   p.tiles_m = (int32_t)((g.rows_a + C::kBM - 1) / C::kBM);
   p.tiles_n = (int32_t)((g.rows_b + BN - 1) / BN);
-  p.d = reinterpret_cast<__nv_bfloat16*>(g.d);
-  p.ldd = g.ldd;
   const int tiles = p.tiles_m * p.tiles_n;
   const int clusters = tiles < max_clusters[dev_id] ? tiles : max_clusters[dev_id];
   cfg.gridDim = dim3(CG * clusters);
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, p) != cudaSuccess) return PURO_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, md, p) != cudaSuccess) return PURO_ERR_CUDA;
   return launch_status();
 }
 

@@ -34,7 +34,7 @@ M_TOKENS = 8192
 # dram__bytes_read.sum + dram__bytes_write.sum of one GEMM launch (fprop, QKV
 # layer) from the ncu capture summarised in profiles/; None until captured
 # for the current kernel.
-GEMM_TRAFFIC_BYTES = 25215232  # QKV fprop launch, profiles/gemm_block_scaled_attn_proj_qkv_fprop.md
+GEMM_TRAFFIC_BYTES = 23336192 + 6405632  # profiles/gemm_block_scaled_attn_proj_qkv_fprop.md
 
 
 def _peaks():
@@ -55,6 +55,7 @@ def _parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ceiling", action="store_true")
     return ap.parse_args()
 
 
@@ -282,6 +283,10 @@ def run_ours(args):
             e2e["ms_per_step"] = float(t.item())
         e2e["value"] = round(gemm_flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12, 2)
 
+    ceiling = None
+    if rank == 0 and not args.no_ceiling:
+        ceiling = fp8_ceiling(wl, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
@@ -338,9 +343,67 @@ def run_ours(args):
                            "ms_per_step": round(e2e["ms_per_step"], 3)}
         if cpu is not None:
             line["cpu_baseline"] = cpu
+        if ceiling is not None:
+            if "tflops_step_shapes" in ceiling:
+                ceiling["gemm_vs_library_same_shapes"] = round(gemm_tf / ceiling["tflops_step_shapes"], 3)
+            line["fp8_library_ceiling"] = ceiling
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def fp8_ceiling(wl, dev):
+    """Library FP8 tensor-core throughput on this GPU, for context: cuBLASLt's
+    MXFP8 GEMM (E4M3 operands, UE8M0 scales per 1x32 block, BF16 out) through
+    torch's scaled_mm, at 8192^3 and at the six GEMM shapes of the step.  Not
+    the same scaling granularity as the path (1x128 / 128x128), so it is a
+    ceiling estimate, not a comparison arm.  None if unavailable."""
+    import torch
+    import torch.nn.functional as F
+    if not hasattr(F, "scaled_mm") or not hasattr(torch, "float8_e8m0fnu"):
+        return None
+
+    def rup(a, b):
+        return (a + b - 1) // b * b
+
+    def timed(m, n, k, reps=20):
+        a = torch.full((m, k), 1.0, device=dev).to(torch.float8_e4m3fn)
+        b = torch.full((n, k), 1.0, device=dev).to(torch.float8_e4m3fn)
+        sa = torch.full((rup(m, 128) * rup(k // 32, 4),), 127, dtype=torch.uint8,
+                        device=dev).view(torch.float8_e8m0fnu)
+        sb = torch.full((rup(n, 128) * rup(k // 32, 4),), 127, dtype=torch.uint8,
+                        device=dev).view(torch.float8_e8m0fnu)
+
+        def f():
+            return F.scaled_mm(a, b.t(), sa, F.ScalingType.BlockWise1x32, sb,
+                               F.ScalingType.BlockWise1x32,
+                               swizzle_a=F.SwizzleType.SWIZZLE_32_4_4,
+                               swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                               output_dtype=torch.bfloat16)
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for s0, s1 in ev:
+            s0.record(); f(); s1.record()
+        torch.cuda.synchronize()
+        ms = sorted(s0.elapsed_time(s1) for s0, s1 in ev)[reps // 2]
+        return ms
+
+    try:
+        ms = timed(8192, 8192, 8192)
+        peak = 2.0 * 8192 ** 3 / (ms * 1e-3) / 1e12
+        tot_ms, tot_flops = 0.0, 0
+        for L in wl.layers:
+            for (m, n, k) in ((L.m, L.n, L.k), (L.m, L.k, L.n), (L.n, L.k, L.m)):
+                tot_ms += timed(m, n, k)
+                tot_flops += 2 * m * n * k
+        return {"source": "cuBLASLt MXFP8 via torch scaled_mm (1x32 UE8M0 scales, BF16 out)",
+                "tflops_8192cube": round(peak, 1),
+                "tflops_step_shapes": round(tot_flops / (tot_ms * 1e-3) / 1e12, 1)}
+    except Exception as e:  # noqa: BLE001  (library path missing on this build)
+        return {"unavailable": str(e).splitlines()[0][:160]}
 
 
 def run_e2e(wl, dev, K, warmup):

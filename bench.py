@@ -56,6 +56,7 @@ def _parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-ceiling", action="store_true")
+    ap.add_argument("--no-bf16", action="store_true")
     return ap.parse_args()
 
 
@@ -287,6 +288,19 @@ def run_ours(args):
     if rank == 0 and not args.no_ceiling:
         ceiling = fp8_ceiling(wl, dev)
 
+    bf16 = None
+    if not args.no_bf16:
+        bms = bf16_step_ms(step, min(K, 200))
+        if world > 1:
+            t = torch.tensor([bms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            bms = float(t.item())
+        bf16 = {"ms_per_step": round(bms, 4),
+                "tflops": round(gemm_flops / (bms * 1e-3) / 1e12, 1),
+                "fp8_speedup": round(bms / ms_per_step, 3),
+                "what": "same step in BF16 via torch.matmul (cuBLAS), no quantization; "
+                        "fp8_speedup = BF16 step time / FP8 step time (quantizers included)"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
@@ -343,6 +357,9 @@ def run_ours(args):
                            "ms_per_step": round(e2e["ms_per_step"], 3)}
         if cpu is not None:
             line["cpu_baseline"] = cpu
+        if bf16 is not None:
+            line["bf16_comparison"] = bf16
+            line["mfu_accounting"] = mfu_accounting(value / world, bf16["tflops"], peaks)
         if ceiling is not None:
             if "tflops_step_shapes" in ceiling:
                 ceiling["gemm_vs_library_same_shapes"] = round(gemm_tf / ceiling["tflops_step_shapes"], 3)
@@ -350,6 +367,69 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def bf16_step_ms(step, K):
+    """The same linear step in BF16 through cuBLAS (torch.matmul): per layer
+    Y = X W^T, dX = dY W, dW = dY^T X, on the same rotating device input sets,
+    K steps captured in one CUDA graph and timed with device events.  This is
+    the FP8-vs-BF16 comparison of the pages' throughput claim, taken at the
+    level of the linear layer."""
+    import torch
+    outs = []
+    for (x, w, dy) in step.sets[0]:
+        outs.append((torch.empty((x.shape[0], w.shape[0]), dtype=torch.bfloat16, device=x.device),
+                     torch.empty_like(x), torch.empty_like(w)))
+
+    def one(i):
+        for (x, w, dy), (y, dx, dw) in zip(step.sets[i % len(step.sets)], outs):
+            torch.matmul(x, w.t(), out=y)
+            torch.matmul(dy, w, out=dx)
+            torch.matmul(dy.t(), x, out=dw)
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True, external=True)
+    t1 = torch.cuda.Event(enable_timing=True, external=True)
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cs):
+        with torch.cuda.graph(g, stream=cs):
+            t0.record()
+            for i in range(K):
+                one(i)
+            t1.record()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / K
+    del g
+    return ms
+
+
+def mfu_accounting(fp8_tflops, bf16_tflops, peaks):
+    """Mixed-precision MFU bookkeeping with the pages' weighting: 72 % of a
+    step's FLOPs in FP8 linear layers, 28 % in BF16.  The effective peak is the
+    time-weighted (harmonic) mean P_eff = (0.72/P_fp8 + 0.28/P_bf16)^-1; the
+    projected throughput combines the measured FP8 linear-layer rate with the
+    measured BF16 cuBLAS rate on the same shapes for the BF16 share."""
+    f8, bf = 0.72, 0.28
+    nominal = {"fp8": 4500.0, "bf16": 2250.0}
+    measured = {"fp8": 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "bf16": peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])}
+    proj = 1.0 / (f8 / fp8_tflops + bf / bf16_tflops)
+    out = {"fp8_share": f8, "bf16_share": bf,
+           "fp8_tflops_measured": round(fp8_tflops, 1), "bf16_tflops_measured": round(bf16_tflops, 1),
+           "projected_tflops": round(proj, 1)}
+    for name, pk in (("nominal", nominal), ("measured", measured)):
+        peff = 1.0 / (f8 / pk["fp8"] + bf / pk["bf16"])
+        out["p_eff_%s" % name] = round(peff, 1)
+        out["mfu_vs_%s" % name] = round(proj / peff, 4)
+    return out
 
 
 def fp8_ceiling(wl, dev):
@@ -367,8 +447,11 @@ def fp8_ceiling(wl, dev):
         return (a + b - 1) // b * b
 
     def timed(m, n, k, reps=20):
-        a = torch.full((m, k), 1.0, device=dev).to(torch.float8_e4m3fn)
-        b = torch.full((n, k), 1.0, device=dev).to(torch.float8_e4m3fn)
+        # random operands: constant ones draw less power and run at clocks a
+        # real GEMM does not keep (measured: 4.0 vs 2.6 PF/s at 8192^3)
+        g = torch.Generator(device=dev).manual_seed(7)
+        a = (torch.randn((m, k), device=dev, generator=g) * 4).to(torch.float8_e4m3fn)
+        b = (torch.randn((n, k), device=dev, generator=g) * 4).to(torch.float8_e4m3fn)
         sa = torch.full((rup(m, 128) * rup(k // 32, 4),), 127, dtype=torch.uint8,
                         device=dev).view(torch.float8_e8m0fnu)
         sb = torch.full((rup(n, 128) * rup(k // 32, 4),), 127, dtype=torch.uint8,

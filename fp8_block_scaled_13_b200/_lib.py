@@ -32,6 +32,7 @@ EXPORTS = (
     "puro_fp8_gemm_fprop",
     "puro_fp8_gemm_dgrad",
     "puro_fp8_gemm_wgrad",
+    "puro_fp8_gemm_wgrad_f32",
     "puro_fp8_device_status",
     "puro_fp8_status_string",
     "puro_fp8_test_bounded_wait",
@@ -64,6 +65,7 @@ def load() -> ctypes.CDLL:
     lib.puro_fp8_gemm_fprop.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
     lib.puro_fp8_gemm_dgrad.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
     lib.puro_fp8_gemm_wgrad.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
+    lib.puro_fp8_gemm_wgrad_f32.argtypes = [P, I, P, P, I, P, P, I, I, I, I, INT, P]
     lib.puro_fp8_device_status.argtypes = [P]
     lib.puro_fp8_status_string.argtypes = [INT]
     lib.puro_fp8_status_string.restype = ctypes.c_char_p
@@ -104,6 +106,12 @@ def puro_fp8_gemm_dgrad(qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, n, 
 def puro_fp8_gemm_wgrad(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k, stream) -> int:
     return load().puro_fp8_gemm_wgrad(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k,
                                       stream)
+
+
+def puro_fp8_gemm_wgrad_f32(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k, accumulate,
+                            stream) -> int:
+    return load().puro_fp8_gemm_wgrad_f32(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k,
+                                          accumulate, stream)
 
 
 def puro_fp8_device_status(stream) -> int:

@@ -38,11 +38,13 @@
 //               release the stage in both CTAs and to publish the tile.
 //   warps 2-9 : epilogue -- warp w reads TMEM lanes 32*(w%4)..+31 (tile rows)
 //               and one half of the columns, releases the accumulator as soon
-//               as its loads completed, then converts to BF16 and writes the
-//               rows through shared memory, 32 columns at a time, with TMA
-//               tensor stores (64-byte row segments; one thread per row
-//               storing straight to global memory touched 32 lines per
-//               instruction and was the throughput limit of the kernel).
+//               as its loads completed, then writes the rows through shared
+//               memory with TMA tensor stores, 64-byte row segments at a time
+//               (32 BF16 or 16 FP32 columns; one thread per row storing
+//               straight to global memory touched 32 lines per instruction and
+//               was the throughput limit of the kernel).  Output kinds: BF16
+//               (RNE), FP32, or FP32 added into the existing output by TMA
+//               reduce-add (accumulation into an FP32 gradient buffer).
 //
 // TMEM (512 columns) holds two accumulators, so the MMAs of the next tile
 // overlap the epilogue of the previous one.  With BN = 256 the two 256-column
@@ -76,6 +78,9 @@ struct GemmParams {
 #ifndef PURO_GEMM_EPI_BUFS
 #define PURO_GEMM_EPI_BUFS 1
 #endif
+
+// Output of the GEMM: D = AB^T as BF16, as FP32, or D += AB^T in FP32.
+enum GemmOut : int { kOutBf16 = 0, kOutF32 = 1, kOutF32Add = 2 };
 
 template <int CG, int BN, int BK>
 struct GemmCfg {
@@ -138,7 +143,7 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
          (1ull << 46) | (4ull << 61);
 }
 
-template <int CG, int BN, int BK>
+template <int CG, int BN, int BK, int OUT>
 __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     gemm_block_scaled_kernel(const __grid_constant__ CUtensorMap tm_a,
                              const __grid_constant__ CUtensorMap tm_b,
@@ -352,23 +357,30 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader<CG>(&acce[acc]);
-      // BF16 rows through this warp's staging buffers: lane = row, 64 bytes
-      // (32 columns) per chunk; one TMA store per chunk writes 32 rows x 64 B
+      // rows through this warp's staging buffers: lane = row, 64 bytes (32 BF16
+      // or 16 FP32 columns) per chunk; one TMA store (or reduce-add) per chunk
+      // writes 32 rows x 64 B
+      constexpr int kCC = (OUT == kOutBf16) ? 32 : 16;  // columns per chunk
       const int row0 = tm * C::kBM + 128 * (int)rank + sp * 32;
       const int gcol = tn * BN + half * C::kEpiCols;
       if (row0 < p.rows_a) {
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-          if (gcol + c * 32 < p.rows_b) {
+        for (int c = 0; c < C::kEpiCols / kCC; ++c) {
+          if (gcol + c * kCC < p.rows_b) {
             uint8_t* buf = ebuf + (ebufc % C::kEpiBufs) * C::kEpiChunkBytes;
             if (lane == 0) bulk_wait_group_read<C::kEpiBufs - 1>();
             __syncwarp();
             uint32_t pk[16];
+            if (OUT == kOutBf16) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[c * 32 + 2 * e]),
-                                                       __uint_as_float(r[c * 32 + 2 * e + 1]));
-              pk[e] = *reinterpret_cast<uint32_t*>(&h);
+              for (int e = 0; e < 16; ++e) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[c * 32 + 2 * e]),
+                                                         __uint_as_float(r[c * 32 + 2 * e + 1]));
+                pk[e] = *reinterpret_cast<uint32_t*>(&h);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pk[e] = r[c * 16 + e];
             }
             uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64);
 #pragma unroll
@@ -377,7 +389,10 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tm_d, buf, gcol + c * 32, row0);
+              if (OUT == kOutF32Add)
+                tma_reduce_add_2d(&tm_d, buf, gcol + c * kCC, row0);
+              else
+                tma_store_2d(&tm_d, buf, gcol + c * kCC, row0);
               bulk_commit_group();
             }
             ++ebufc;

@@ -166,11 +166,12 @@ struct GemmArgs {
   const void* sfa;                 // blocked, rows_a x ceil(K/128) groups
   const void* b;    int64_t ldb;   // E4M3 [rows_b, K]
   const void* sfb;                 // blocked, rows_b x ceil(K/128) groups
-  void* d; int64_t ldd;
+  void* d; int64_t ldd;             // output [rows_a, rows_b], ldd elements per row
   int64_t rows_a, rows_b, k;
+  int out;                          // puro::GemmOut
 };
 
-template <int CG, int BN, int BK>
+template <int CG, int BN, int BK, int OUT>
 int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
   using C = puro::GemmCfg<CG, BN, BK>;
   CUtensorMap ma, mb, msa, msb;
@@ -181,19 +182,22 @@ int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
   if ((st = make_map_u8(&mb, g.b, g.k, g.rows_b, g.ldb, BK, C::kBNC, sw)) != PURO_OK) return st;
   if ((st = make_map_scales(&msa, g.sfa, g.rows_a, kb, 1)) != PURO_OK) return st;
   if ((st = make_map_scales(&msb, g.sfb, g.rows_b, kb, C::kNB)) != PURO_OK) return st;
-  // BF16 output [rows_a, rows_b], row stride ldd elements; 32 x 32 store boxes
+  // output [rows_a, rows_b], row stride ldd elements; store boxes of 32 rows
+  // x 64 bytes (32 BF16 or 16 FP32 columns)
   CUtensorMap md;
   {
+    const bool f32 = OUT != puro::kOutBf16;
     cuuint64_t dims[2] = {(cuuint64_t)g.rows_b, (cuuint64_t)g.rows_a};
-    cuuint64_t strides[1] = {(cuuint64_t)g.ldd * 2};
-    cuuint32_t box[2] = {32, 32};
+    cuuint64_t strides[1] = {(cuuint64_t)g.ldd * (f32 ? 4 : 2)};
+    cuuint32_t box[2] = {f32 ? 16u : 32u, 32};
     cuuint32_t estr[2] = {1, 1};
-    if (g_encode(&md, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.d, dims, strides, box, estr,
+    if (g_encode(&md, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                 g.d, dims, strides, box, estr,
                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return PURO_ERR_CUDA;
   }
-  auto kern = puro::gemm_block_scaled_kernel<CG, BN, BK>;
+  auto kern = puro::gemm_block_scaled_kernel<CG, BN, BK, OUT>;
   static int max_clusters[kMaxDevices] = {};
   int dev_id = 0;
   cudaGetDevice(&dev_id);
@@ -240,13 +244,24 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
   if ((st = get_encoder()) != PURO_OK) return st;
   if (g.rows_a == 0 || g.rows_b == 0) return PURO_OK;
   if (g.k == 0) {
-    // empty reduction: the product is exactly zero
-    if (cudaMemset2DAsync(g.d, (size_t)g.ldd * 2, 0, (size_t)g.rows_b * 2, (size_t)g.rows_a,
+    // empty reduction: the product is exactly zero (nothing to add when accumulating)
+    if (g.out == puro::kOutF32Add) return PURO_OK;
+    const size_t es = g.out == puro::kOutBf16 ? 2 : 4;
+    if (cudaMemset2DAsync(g.d, (size_t)g.ldd * es, 0, (size_t)g.rows_b * es, (size_t)g.rows_a,
                           stream) != cudaSuccess)
       return PURO_ERR_CUDA;
     return PURO_OK;
   }
-  return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN, PURO_GEMM_BK>(g, dev, stream);
+  switch (g.out) {
+    case puro::kOutBf16:
+      return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN, PURO_GEMM_BK, puro::kOutBf16>(g, dev, stream);
+    case puro::kOutF32:
+      return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN, PURO_GEMM_BK, puro::kOutF32>(g, dev, stream);
+    case puro::kOutF32Add:
+      return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN, PURO_GEMM_BK, puro::kOutF32Add>(g, dev, stream);
+    default:
+      return PURO_ERR_LAYOUT;
+  }
 }
 
 // Shape/alignment checks shared by the three GEMMs.
@@ -373,7 +388,7 @@ int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx, const voi
     if (!sx || !sw_fwd) return PURO_ERR_NULL;
     if (!aligned16(sx) || !aligned16(sw_fwd)) return PURO_ERR_ALIGN;
   }
-  GemmArgs g{qx, ld_qx, sx, qw, ld_qw, sw_fwd, y, ld_y, m, n, k};
+  GemmArgs g{qx, ld_qx, sx, qw, ld_qw, sw_fwd, y, ld_y, m, n, k, puro::kOutBf16};
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
@@ -391,7 +406,7 @@ int puro_fp8_gemm_dgrad(const void* qdy, int64_t ld_qdy, const void* sdy, const 
     if (!sdy || !sw_bwd) return PURO_ERR_NULL;
     if (!aligned16(sdy) || !aligned16(sw_bwd)) return PURO_ERR_ALIGN;
   }
-  GemmArgs g{qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, k, n};
+  GemmArgs g{qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, k, n, puro::kOutBf16};
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
@@ -409,7 +424,27 @@ int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* sdyt, con
     if (!sdyt || !sxt) return PURO_ERR_NULL;
     if (!aligned16(sdyt) || !aligned16(sxt)) return PURO_ERR_ALIGN;
   }
-  GemmArgs g{qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, n, k, m};
+  GemmArgs g{qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, n, k, m, puro::kOutBf16};
+  return launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+int puro_fp8_gemm_wgrad_f32(const void* qdyt, int64_t ld_qdyt, const void* sdyt, const void* qxt,
+                            int64_t ld_qxt, const void* sxt, void* dw, int64_t ld_dw, int64_t m,
+                            int64_t n, int64_t k, int accumulate, void* stream) {
+  if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
+  if (n % 128 || k % 128) return PURO_ERR_SHAPE;
+  if (accumulate != 0 && accumulate != 1) return PURO_ERR_LAYOUT;
+  if (n == 0 || k == 0) return PURO_OK;
+  int r;
+  if ((r = check_mat(dw, ld_dw, k, 4)) != PURO_OK) return r;
+  if (m > 0) {
+    if ((r = check_mat(qdyt, ld_qdyt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
+    if ((r = check_mat(qxt, ld_qxt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
+    if (!sdyt || !sxt) return PURO_ERR_NULL;
+    if (!aligned16(sdyt) || !aligned16(sxt)) return PURO_ERR_ALIGN;
+  }
+  GemmArgs g{qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, n, k, m,
+             accumulate ? puro::kOutF32Add : puro::kOutF32};
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 

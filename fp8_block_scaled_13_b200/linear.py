@@ -149,13 +149,31 @@ def gemm_dgrad(dyq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) 
     return out
 
 
-def gemm_wgrad(dyq: QuantAct, xq: QuantAct, out: torch.Tensor | None = None) -> torch.Tensor:
-    """dW = dY^T X [n, k] BF16 from the COLWISE quantizations of dY and X."""
+def gemm_wgrad(dyq: QuantAct, xq: QuantAct, out: torch.Tensor | None = None,
+               accumulate: bool = False) -> torch.Tensor:
+    """dW = dY^T X [n, k] from the COLWISE quantizations of dY and X.
+
+    `out` BF16 (default) or FP32.  With an FP32 `out` and accumulate=True the
+    product is added to it (dW += dY^T X, an FP32 gradient buffer); only the
+    FP32 output accumulates."""
     m, n, k = dyq.rows, dyq.cols, xq.cols
     if xq.rows != m:
         raise ValueError("dY and X have different token counts")
     if out is None:
+        if accumulate:
+            raise ValueError("accumulate=True needs the FP32 buffer to add into")
         out = torch.empty((n, k), dtype=torch.bfloat16, device=dyq.qt.device)
+    if tuple(out.shape) != (n, k) or out.stride(1) != 1:
+        raise ValueError("out must be a row-major [n, k] tensor")
+    if out.dtype == torch.float32:
+        st = _lib.puro_fp8_gemm_wgrad_f32(
+            dyq.qt.data_ptr(), dyq.qt.stride(0), dyq.st.data_ptr(),
+            xq.qt.data_ptr(), xq.qt.stride(0), xq.st.data_ptr(),
+            out.data_ptr(), out.stride(0), m, n, k, 1 if accumulate else 0, _stream())
+        _check(st, "puro_fp8_gemm_wgrad_f32")
+        return out
+    if out.dtype != torch.bfloat16 or accumulate:
+        raise ValueError("out must be BF16, or FP32 (required for accumulate=True)")
     st = _lib.puro_fp8_gemm_wgrad(
         dyq.qt.data_ptr(), dyq.qt.stride(0), dyq.st.data_ptr(),
         xq.qt.data_ptr(), xq.qt.stride(0), xq.st.data_ptr(),
@@ -176,7 +194,14 @@ def linear_forward(x: torch.Tensor, w: torch.Tensor):
     return gemm_fprop(xq, wq), xq, wq
 
 
-def linear_backward(dy: torch.Tensor, xq: QuantAct, wq: QuantWeight):
-    """Quantize dY both ways, then dX = dY W and dW = dY^T X.  Returns (dx, dw)."""
+def linear_backward(dy: torch.Tensor, xq: QuantAct, wq: QuantWeight,
+                    main_grad: torch.Tensor | None = None):
+    """Quantize dY both ways, then dX = dY W and dW = dY^T X.  Returns (dx, dw).
+
+    With `main_grad` (FP32 [n, k]) the weight gradient is added into it
+    (gradient accumulation across micro-batches) and returned as dw."""
     dyq = quant_act(dy, "both")
-    return gemm_dgrad(dyq, wq), gemm_wgrad(dyq, xq)
+    dx = gemm_dgrad(dyq, wq)
+    if main_grad is not None:
+        return dx, gemm_wgrad(dyq, xq, out=main_grad, accumulate=True)
+    return dx, gemm_wgrad(dyq, xq)

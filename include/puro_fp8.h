@@ -174,6 +174,27 @@ PURO_API int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* 
                                  void* stream);
 
 /*
+ * puro_fp8_gemm_wgrad_f32 -- the weight-gradient GEMM with an FP32 result:
+ *   accumulate == 0 : dW  = dY^T X
+ *   accumulate == 1 : dW += dY^T X   (accumulation into an FP32 gradient
+ *                                     buffer across micro-batches)
+ * The pages keep gradients in FP32 while the three linear-layer GEMMs run in
+ * E4M3 (paperlayer.ai Appendix C, "Production Training Details", the FP8
+ * implementation pipeline; micro-batch size 2 under a 1,536-sequence global
+ * batch in the same appendix, hence the accumulation).
+ * Operands as puro_fp8_gemm_wgrad.  dw : FP32 [n, k], row stride ld_dw
+ * elements (ld_dw * 4 a multiple of 16 bytes), caller-owned, 16-byte aligned.
+ * Each element receives exactly one FP32 store or one FP32 add per call (the
+ * add is done by the memory system, as a TMA reduce-add), so repeated calls
+ * give the same result for the same inputs.  m == 0: dW = 0, or unchanged
+ * when accumulating.  accumulate other than 0/1 -> PURO_ERR_LAYOUT.
+ */
+PURO_API int puro_fp8_gemm_wgrad_f32(const void* qdyt, int64_t ld_qdyt, const void* sdyt,
+                                     const void* qxt, int64_t ld_qxt, const void* sxt,
+                                     void* dw, int64_t ld_dw, int64_t m, int64_t n, int64_t k,
+                                     int accumulate, void* stream);
+
+/*
  * puro_fp8_device_status -- synchronizes `stream`, then returns and clears the
  * library's device error word for the current device: PURO_OK, or
  * PURO_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the last

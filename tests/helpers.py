@@ -65,3 +65,19 @@ def assert_gemm_close(got, ref64, oracle, what=""):
     assert rel <= 1e-3, "%s: relative Frobenius error %.3g > 1e-3" % (what, rel)
     assert excess <= 0.0, "%s: an element exceeds 4e-3*rms + 1 ulp by %.3g" % (what, excess)
     return rel
+
+
+def assert_f32_close(got, ref64: np.ndarray, init=None, what=""):
+    """FP32-output GEMM check: relative Frobenius error <= 1e-3 of the FP64
+    product, and every element within 4e-3 * rms(product) + 1 FP32 ulp of the
+    expected value (init + product when the output was accumulated into)."""
+    g = got.detach().cpu().numpy().astype(np.float64)
+    exp = ref64 if init is None else np.asarray(init, dtype=np.float64) + ref64
+    den = np.linalg.norm(ref64)
+    rel = np.linalg.norm(g - exp) / den if den > 0 else np.linalg.norm(g - exp)
+    assert rel <= 1e-3, "%s: relative Frobenius error %.3g > 1e-3" % (what, rel)
+    rms = np.sqrt(np.mean(ref64 ** 2)) if ref64.size else 0.0
+    ulp = np.spacing(np.abs(exp).astype(np.float32)).astype(np.float64)
+    excess = np.abs(g - exp) - (4e-3 * rms + ulp)
+    assert excess.max() <= 0.0, "%s: an element exceeds the tolerance by %.3g" % (what, excess.max())
+    return rel

@@ -111,9 +111,25 @@ def test_gemm_argument_errors(lib, fn, args, code):
     assert f(*args, None) == code
 
 
+@pytest.mark.parametrize("args,code", [
+    # (qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k, accumulate)
+    ((A, 64, A, A, 64, A, A, 256, 64, 256, 256, 2), -4),     # accumulate flag not 0/1
+    ((A, 64, A, A, 64, A, A, 258, 64, 256, 256, 0), -2),     # ld_dw * 4 not a multiple of 16
+    ((A, 64, A, A, 64, A, A, 128, 64, 256, 256, 1), -3),     # ld_dw < k
+    ((A, 64, A, A, 64, A, A, 256, 64, 200, 256, 0), -3),     # n % 128
+    ((A, 64, A, A, 64, A, A + 8, 256, 64, 256, 256, 1), -2), # dw misaligned
+    ((A, 48, A, A, 64, A, A, 256, 64, 256, 256, 0), -3),     # ld_qdyt < m
+    ((A, 64, None, A, 64, A, A, 256, 64, 256, 256, 1), -1),  # sdyt null
+])
+def test_wgrad_f32_argument_errors(lib, args, code):
+    assert lib.puro_fp8_gemm_wgrad_f32(*args, None) == code
+
+
 def test_gemm_empty_is_noop(lib):
     assert lib.puro_fp8_gemm_fprop(None, 0, None, None, 0, None, None, 0, 0, 256, 256, None) == 0
     assert lib.puro_fp8_gemm_wgrad(None, 0, None, None, 0, None, None, 0, 64, 0, 256, None) == 0
+    assert lib.puro_fp8_gemm_wgrad_f32(None, 0, None, None, 0, None, None, 0, 64, 0, 256, 1,
+                                       None) == 0
 
 
 @pytest.mark.parametrize("rows,groups,want", [

@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_gemm_close, np_u8, unblock
+from helpers import assert_f32_close, assert_gemm_close, np_u8, unblock
 
 pytestmark = pytest.mark.gpu
 
@@ -81,6 +81,12 @@ def _check_layer(fp8, oracle_mod, L, seed):
     cols = _sample(n, N_ROWS, seed + 2)
     ref = oracle_mod.linear_wgrad(L.dy[:, cols].contiguous(), L.x)
     assert_gemm_close(dw[cols.tolist()], ref, oracle_mod, "%s wgrad" % L.name)
+    # the FP32 gradient buffer path: accumulate into an initialised buffer
+    init = torch.full((n, k), 0.25, dtype=torch.float32, device=dev)
+    fp8.gemm_wgrad(dyq, xq, out=init, accumulate=True)
+    torch.cuda.synchronize()
+    assert fp8.device_status() == 0
+    assert_f32_close(init[cols.tolist()], ref, np.full(ref.shape, 0.25), "%s wgrad += FP32" % L.name)
 
 
 @pytest.mark.parametrize("name", ["single_fprop"])

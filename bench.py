@@ -57,6 +57,9 @@ def _parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-ceiling", action="store_true")
     ap.add_argument("--no-bf16", action="store_true")
+    ap.add_argument("--accum", type=int, default=64,
+                    help="micro-batch steps per gradient exchange (the pages: 1536 sequences / "
+                         "(DP 12 x MBS 2) = 64)")
     return ap.parse_args()
 
 
@@ -124,6 +127,7 @@ class Step:
     def __init__(self, wl, dev, n_sets=3):
         import torch
         import fp8_block_scaled_13_b200 as fp8
+        from fp8_block_scaled_13_b200.dp import MainGrads
         self.fp8 = fp8
         self.torch = torch
         self.layers = wl.layers
@@ -139,8 +143,10 @@ class Step:
             dyq = fp8.quant_act(dy, "both")
             y = torch.empty((x.shape[0], w.shape[0]), dtype=torch.bfloat16, device=dev)
             dx = torch.empty_like(x)
-            dw = torch.empty_like(w)
-            self.out.append((xq, wq, dyq, y, dx, dw))
+            self.out.append((xq, wq, dyq, y, dx))
+        # FP32 weight gradients of both layers in one buffer: every step adds
+        # its dW into it (one micro-batch of gradient accumulation)
+        self.grads = MainGrads([(w.shape[0], w.shape[1]) for (_, w, _) in self.sets[0]], device=dev)
         torch.cuda.synchronize()
         self.names = []
         for L in wl.layers:
@@ -156,13 +162,21 @@ class Step:
             if ev is not None:
                 next(ev).record()
 
-        for (x, w, dy), (xq, wq, dyq, y, dx, dw) in zip(self.sets[set_idx], self.out):
+        for li, ((x, w, dy), (xq, wq, dyq, y, dx)) in enumerate(zip(self.sets[set_idx], self.out)):
             mark(); fp8.quant_weight(w, transpose=True, out=wq); mark()
             mark(); fp8.quant_act(x, "both", out=xq); mark()
             mark(); fp8.gemm_fprop(xq, wq, out=y); mark()
             mark(); fp8.quant_act(dy, "both", out=dyq); mark()
             mark(); fp8.gemm_dgrad(dyq, wq, out=dx); mark()
-            mark(); fp8.gemm_wgrad(dyq, xq, out=dw); mark()
+            mark(); fp8.gemm_wgrad(dyq, xq, out=self.grads[li], accumulate=True); mark()
+
+    def sync_grads(self, world):
+        """End of a gradient-accumulation window: exchange the FP32 weight
+        gradients across the data-parallel ranks (all-reduce, averaged), then
+        clear them as the optimizer step would."""
+        if world > 1:
+            self.grads.all_reduce_(average=True)
+        self.grads.zero_()
 
 
 def _unit_costs(wl):
@@ -202,40 +216,53 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError("device status %d after warm-up" % status)
 
-    # The K timed steps are captured once into a CUDA graph (kernel arguments,
-    # including the TMA descriptors, are baked in), so the timed region holds
-    # device work only.  A second graph of the same K steps carries an event
-    # pair around every launch for the per-kernel breakdown; it is replayed
-    # separately because event nodes between kernels also cut the programmatic
-    # (PDL) edges that let a kernel's prologue overlap its predecessor's tail.
+    # The timed steps run as CUDA graphs (kernel arguments, including the TMA
+    # descriptors, are baked in), so the timed region holds device work only:
+    # a graph of `accum` micro-batch steps is replayed, and after each window
+    # the FP32 weight gradients are exchanged across the ranks (NCCL
+    # all-reduce, outside the graph) and cleared; exactly K steps in all (a
+    # shorter graph covers the remainder).  A separate graph with an event
+    # pair around every launch gives the per-kernel breakdown; it is replayed
+    # on its own because event nodes between kernels also cut the
+    # programmatic (PDL) edges that let a kernel's prologue overlap its
+    # predecessor's tail.
     K = args.steps
+    A = max(1, min(args.accum, K))
+    windows = [A] * (K // A) + ([K % A] if K % A else [])
     nl = step.launches_per_step
-    t_start = torch.cuda.Event(enable_timing=True, external=True)
-    t_end = torch.cuda.Event(enable_timing=True, external=True)
+    K_inst = min(K, 100)
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * nl)]
-          for _ in range(K)]
-    graph = torch.cuda.CUDAGraph()
+          for _ in range(K_inst)]
+    graphs = {}
     graph_inst = torch.cuda.CUDAGraph()
     cap_stream = torch.cuda.Stream()
     cap_stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(cap_stream):
-        with torch.cuda.graph(graph, stream=cap_stream):
-            t_start.record()
-            for i in range(K):
-                step.run(i % len(step.sets))
-            t_end.record()
+        for n in sorted(set(windows)):
+            graphs[n] = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graphs[n], stream=cap_stream):
+                for i in range(n):
+                    step.run(i % len(step.sets))
         with torch.cuda.graph(graph_inst, stream=cap_stream):
-            for i in range(K):
+            for i in range(K_inst):
                 step.run(i % len(step.sets), ev[i])
     torch.cuda.synchronize()
-    graph.replay()  # untimed first replays of the instantiated graphs
+    for g in graphs.values():  # untimed first replays of the instantiated graphs
+        g.replay()
     graph_inst.replay()
+    step.sync_grads(world)
     torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        graph.replay()
+        t_start.record()
+        for n in windows:
+            graphs[n].replay()
+            step.sync_grads(world)
+        t_end.record()
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -249,7 +276,7 @@ def run_ours(args):
 
     total_ms = t_start.elapsed_time(t_end)
     per_launch = {name: [] for name in step.names}
-    for i in range(K):
+    for i in range(K_inst):
         for j, name in enumerate(step.names):
             per_launch[name].append(ev[i][2 * j].elapsed_time(ev[i][2 * j + 1]))
     ms_per_step = total_ms / K
@@ -257,7 +284,7 @@ def run_ours(args):
         t = torch.tensor([ms_per_step], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_per_step = float(t.item())
-    del graph, graph_inst
+    del graphs, graph_inst
 
     peaks, peak_kind = _peaks()
     fp8_peak_tf = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -325,8 +352,11 @@ def run_ours(args):
                 "seed": SEED,
                 "global_batch_tokens": M_TOKENS * world,
                 "l2": "3 rotating input sets of 132 MB each (> 126 MB L2)",
-                "parallelism": "dp%d replicas, no collective" % world,
-                "step": "per layer: quant_weight, quant_act(X), fprop, quant_act(dY), dgrad, wgrad",
+                "parallelism": "dp%d (own batch per rank; FP32 dW all-reduce every %d steps)" % (world, A),
+                "step": "per layer: quant_weight, quant_act(X), fprop, quant_act(dY), dgrad, "
+                        "wgrad added into FP32 main grads",
+                "grad_exchange": "every %d steps: FP32 dW all-reduce across ranks (NCCL) and clear"
+                                 % A,
             },
             "pct_fp8_peak": round(100.0 * value / world / fp8_peak_tf, 1),
             "roofline": {
@@ -348,8 +378,9 @@ def run_ours(args):
             "gpu_launches": step.launches_per_step * K,
             "clocks": clocks,
             "wall_ms_timed_region": round(total_ms, 3),
-            "timing": "K steps replayed as one CUDA graph (device events around it); per-kernel "
-                      "times from a second replay with an event pair around every launch",
+            "timing": "K steps as CUDA graphs of %d steps plus the gradient exchange between them "
+                      "(device events around it all); per-kernel times from a separate replay of %d "
+                      "steps with an event pair around every launch" % (A, K_inst),
         }
         if e2e is not None:
             line["e2e"] = {"value": e2e["value"], "unit": "TFLOP/s",
@@ -491,24 +522,28 @@ def fp8_ceiling(wl, dev):
 
 def run_e2e(wl, dev, K, warmup):
     """Same step through the public API with pinned host inputs/outputs: every
-    step copies X, W, dY in and Y, dX, dW out inside the timed region."""
+    step copies X, W, dY in, runs forward and backward (dW added into the FP32
+    main grads), and copies Y, dX and the main grads back, all inside the
+    timed region."""
     import torch
     import fp8_block_scaled_13_b200 as fp8
+    from fp8_block_scaled_13_b200.dp import MainGrads
 
     host_in = [(L.x.pin_memory(), L.w.pin_memory(), L.dy.pin_memory()) for L in wl.layers]
     host_out = [(torch.empty((L.m, L.n), dtype=torch.bfloat16).pin_memory(),
                  torch.empty((L.m, L.k), dtype=torch.bfloat16).pin_memory(),
-                 torch.empty((L.n, L.k), dtype=torch.bfloat16).pin_memory()) for L in wl.layers]
+                 torch.empty((L.n, L.k), dtype=torch.float32).pin_memory()) for L in wl.layers]
+    grads = MainGrads([(L.n, L.k) for L in wl.layers], device=dev)
     h2d = sum(t.numel() * t.element_size() for tup in host_in for t in tup)
     d2h = sum(t.numel() * t.element_size() for tup in host_out for t in tup)
 
     def one():
-        for (hx, hw, hdy), (hy, hdx, hdw) in zip(host_in, host_out):
+        for li, ((hx, hw, hdy), (hy, hdx, hdw)) in enumerate(zip(host_in, host_out)):
             x = hx.to(dev, non_blocking=True)
             w = hw.to(dev, non_blocking=True)
             dy = hdy.to(dev, non_blocking=True)
             y, xq, wq = fp8.linear_forward(x, w)
-            dx, dw = fp8.linear_backward(dy, xq, wq)
+            dx, dw = fp8.linear_backward(dy, xq, wq, main_grad=grads[li])
             hy.copy_(y, non_blocking=True)
             hdx.copy_(dx, non_blocking=True)
             hdw.copy_(dw, non_blocking=True)

@@ -1,16 +1,18 @@
 """Benchmark of the block-scaled FP8 linear layer hot path on B200.
 
-One step = the whole hot path over one batch of the attention-projection
-workload (M = 8192 tokens, hidden 2048; the fused QKV projection 2048->3072
-and the output projection 2048->2048), for each of the two layers:
+One step = one micro-batch of the attention-projection workload (M = 8192
+tokens, hidden 2048; the fused QKV projection 2048->3072 and the output
+projection 2048->2048), for each of the two layers:
   quant_weight(W) (+ transposed codes), quant_act(X, both), fprop,
-  quant_act(dY, both), dgrad, wgrad.
+  quant_act(dY, both), and one launch computing dgrad and wgrad (dW added
+  into FP32 main grads).
 value = GEMM FLOPs of the step (2*M*N*K per GEMM, three GEMMs per layer)
 divided by the device time of the whole step (quantizers included).
 
-Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-With N > 1 (torchrun) every rank runs its own batch (data-parallel replicas,
-weak scaling); there is no collective in the step.
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--accum A]
+                       [--impl ours|reference]
+With N > 1 (torchrun) every rank runs its own batch (data parallel, weak
+scaling) and every A steps the ranks all-reduce the FP32 weight gradients.
 """
 from __future__ import annotations
 
@@ -34,7 +36,7 @@ M_TOKENS = 8192
 # dram__bytes_read.sum + dram__bytes_write.sum of one GEMM launch (fprop, QKV
 # layer) from the ncu capture summarised in profiles/; None until captured
 # for the current kernel.
-GEMM_TRAFFIC_BYTES = 23336192 + 6405632  # profiles/gemm_block_scaled_attn_proj_qkv_fprop.md
+GEMM_TRAFFIC_BYTES = None  # recaptured after the scheduled-launch change (profiles/)
 
 
 def _peaks():
@@ -151,7 +153,7 @@ class Step:
         self.names = []
         for L in wl.layers:
             self.names += ["%s.quant_weight" % L.name, "%s.quant_x" % L.name, "%s.fprop" % L.name,
-                           "%s.quant_dy" % L.name, "%s.dgrad" % L.name, "%s.wgrad" % L.name]
+                           "%s.quant_dy" % L.name, "%s.dgrad_wgrad" % L.name]
         self.launches_per_step = len(self.names)
 
     def run(self, set_idx, events=None):
@@ -167,8 +169,7 @@ class Step:
             mark(); fp8.quant_act(x, "both", out=xq); mark()
             mark(); fp8.gemm_fprop(xq, wq, out=y); mark()
             mark(); fp8.quant_act(dy, "both", out=dyq); mark()
-            mark(); fp8.gemm_dgrad(dyq, wq, out=dx); mark()
-            mark(); fp8.gemm_wgrad(dyq, xq, out=self.grads[li], accumulate=True); mark()
+            mark(); fp8.gemm_dgrad_wgrad(dyq, wq, xq, dx=dx, dw=self.grads[li], accumulate=True); mark()
 
     def sync_grads(self, world):
         """End of a gradient-accumulation window: exchange the FP32 weight
@@ -187,8 +188,8 @@ def _unit_costs(wl):
         costs["%s.quant_weight" % L.name] = ("bytes", n * k * 2 + 2 * n * k + (n // 128) * (k // 128))
         costs["%s.quant_x" % L.name] = ("bytes", m * k * 2 + 2 * m * k + 2 * m * k // 128)
         costs["%s.quant_dy" % L.name] = ("bytes", m * n * 2 + 2 * m * n + 2 * m * n // 128)
-        for g in ("fprop", "dgrad", "wgrad"):
-            costs["%s.%s" % (L.name, g)] = ("flops", 2 * m * n * k)
+        costs["%s.fprop" % L.name] = ("flops", 2 * m * n * k)
+        costs["%s.dgrad_wgrad" % L.name] = ("flops", 4 * m * n * k)
     return costs
 
 
@@ -353,8 +354,8 @@ def run_ours(args):
                 "global_batch_tokens": M_TOKENS * world,
                 "l2": "3 rotating input sets of 132 MB each (> 126 MB L2)",
                 "parallelism": "dp%d (own batch per rank; FP32 dW all-reduce every %d steps)" % (world, A),
-                "step": "per layer: quant_weight, quant_act(X), fprop, quant_act(dY), dgrad, "
-                        "wgrad added into FP32 main grads",
+                "step": "per layer: quant_weight, quant_act(X), fprop, quant_act(dY), and one "
+                        "launch for dgrad + wgrad (dW added into FP32 main grads)",
                 "grad_exchange": "every %d steps: FP32 dW all-reduce across ranks (NCCL) and clear"
                                  % A,
             },

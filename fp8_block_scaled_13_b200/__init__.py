@@ -8,7 +8,8 @@ libpuro_fp8.so and raises if it is missing.  There is no CPU fallback.
 from __future__ import annotations
 
 _API = ("quant_act", "quant_weight", "blocked_scale_bytes", "gemm_fprop", "gemm_dgrad", "gemm_wgrad",
-        "device_status", "linear_forward", "linear_backward", "QuantAct", "QuantWeight")
+        "gemm_dgrad_wgrad", "device_status", "linear_forward", "linear_backward", "QuantAct",
+        "QuantWeight")
 
 
 def __getattr__(name):

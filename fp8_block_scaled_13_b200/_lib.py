@@ -24,6 +24,9 @@ PURO_ERR_DEVICE_TIMEOUT = -7
 PURO_ROWWISE = 1
 PURO_COLWISE = 2
 PURO_BOTH = 3
+PURO_DW_BF16 = 0
+PURO_DW_F32 = 1
+PURO_DW_F32_ACCUMULATE = 2
 
 EXPORTS = (
     "puro_fp8_blocked_scale_bytes",
@@ -33,6 +36,7 @@ EXPORTS = (
     "puro_fp8_gemm_dgrad",
     "puro_fp8_gemm_wgrad",
     "puro_fp8_gemm_wgrad_f32",
+    "puro_fp8_gemm_dgrad_wgrad",
     "puro_fp8_device_status",
     "puro_fp8_status_string",
     "puro_fp8_test_bounded_wait",
@@ -66,6 +70,8 @@ def load() -> ctypes.CDLL:
     lib.puro_fp8_gemm_dgrad.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
     lib.puro_fp8_gemm_wgrad.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
     lib.puro_fp8_gemm_wgrad_f32.argtypes = [P, I, P, P, I, P, P, I, I, I, I, INT, P]
+    lib.puro_fp8_gemm_dgrad_wgrad.argtypes = [P, I, P, P, I, P, P, I, P, I, P, P, I, P, P, I,
+                                              I, I, I, INT, P]
     lib.puro_fp8_device_status.argtypes = [P]
     lib.puro_fp8_status_string.argtypes = [INT]
     lib.puro_fp8_status_string.restype = ctypes.c_char_p
@@ -112,6 +118,13 @@ def puro_fp8_gemm_wgrad_f32(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m,
                             stream) -> int:
     return load().puro_fp8_gemm_wgrad_f32(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k,
                                           accumulate, stream)
+
+
+def puro_fp8_gemm_dgrad_wgrad(qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, qdyt, ld_qdyt, sdyt,
+                              qxt, ld_qxt, sxt, dw, ld_dw, m, n, k, dw_kind, stream) -> int:
+    return load().puro_fp8_gemm_dgrad_wgrad(qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, qdyt,
+                                            ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k,
+                                            dw_kind, stream)
 
 
 def puro_fp8_device_status(stream) -> int:

@@ -65,12 +65,40 @@
 
 namespace puro {
 
-struct GemmParams {
+// One GEMM of a launch: D [rows_a, rows_b] (through its tm_d tensor map).
+struct GemmProblem {
   int32_t rows_a;   // output rows
   int32_t rows_b;   // output cols
-  int32_t kblocks;  // ceil(K / 128)
-  int32_t tiles_m, tiles_n;  // the BF16 output goes through the tm_d tensor map
+  int32_t kblocks;  // ceil(K / BK)
+  int32_t tiles_m, tiles_n;
 };
+
+constexpr int kMaxSchedClusters = 128;
+constexpr int kMaxSchedUnits = 2048;
+
+// A launch computes one or two independent GEMMs (the data and weight
+// gradients of one layer share a launch).  Its work units are the output tiles:
+// units [0, tiles0) are problem 0's tiles, the rest problem 1's.  Clusters take
+// units either round robin (unit u -> cluster u % clusters) or from a host-made
+// schedule: cluster c runs sched_unit[sched_off[c] .. sched_off[c+1]) in order.
+struct GemmParams {
+  GemmProblem prob[2];
+  int32_t nprob;
+  int32_t tiles0;
+  int32_t units;
+  int32_t sched;
+  uint16_t sched_off[kMaxSchedClusters + 1];
+  uint16_t sched_unit[kMaxSchedUnits];
+};
+
+__device__ __forceinline__ int unit_count(const GemmParams& p, int cluster, int nclusters) {
+  if (p.sched) return (int)p.sched_off[cluster + 1] - (int)p.sched_off[cluster];
+  return cluster < p.units ? (p.units - cluster + nclusters - 1) / nclusters : 0;
+}
+
+__device__ __forceinline__ int unit_at(const GemmParams& p, int cluster, int nclusters, int i) {
+  return p.sched ? (int)p.sched_unit[p.sched_off[cluster] + i] : cluster + i * nclusters;
+}
 
 #ifndef PURO_GEMM_BK
 #define PURO_GEMM_BK 128
@@ -143,13 +171,64 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
          (1ull << 46) | (4ull << 61);
 }
 
-template <int CG, int BN, int BK, int OUT>
+// Epilogue of one warp for one tile: its 32 accumulator rows x kEpiCols
+// columns (in r) go through the warp's staging buffers, 64 bytes per row per
+// chunk (32 BF16 or 16 FP32 columns), one TMA store or reduce-add per chunk.
+template <class C, int OUT>
+__device__ __forceinline__ void epilogue_store(const uint32_t (&r)[C::kEpiCols], const CUtensorMap* tmd,
+                                               uint8_t* ebuf, int& ebufc, int lane, int row0, int gcol,
+                                               int rows_a, int rows_b) {
+  constexpr int kCC = (OUT == kOutBf16) ? 32 : 16;  // columns per chunk
+  if (row0 >= rows_a) return;
+#pragma unroll
+  for (int c = 0; c < C::kEpiCols / kCC; ++c) {
+    if (gcol + c * kCC < rows_b) {
+      uint8_t* buf = ebuf + (ebufc % C::kEpiBufs) * C::kEpiChunkBytes;
+      if (lane == 0) bulk_wait_group_read<C::kEpiBufs - 1>();
+      __syncwarp();
+      uint32_t pk[16];
+      if (OUT == kOutBf16) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[c * 32 + 2 * e]),
+                                                   __uint_as_float(r[c * 32 + 2 * e + 1]));
+          pk[e] = *reinterpret_cast<uint32_t*>(&h);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = r[c * 16 + e];
+      }
+      uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (OUT == kOutF32Add)
+          tma_reduce_add_2d(tmd, buf, gcol + c * kCC, row0);
+        else
+          tma_store_2d(tmd, buf, gcol + c * kCC, row0);
+        bulk_commit_group();
+      }
+      ++ebufc;
+    }
+  }
+}
+
+template <int CG, int BN, int BK, int OUT0, int OUT1>
 __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
-    gemm_block_scaled_kernel(const __grid_constant__ CUtensorMap tm_a,
-                             const __grid_constant__ CUtensorMap tm_b,
-                             const __grid_constant__ CUtensorMap tm_sfa,
-                             const __grid_constant__ CUtensorMap tm_sfb,
-                             const __grid_constant__ CUtensorMap tm_d, const GemmParams p) {
+    gemm_block_scaled_kernel(const __grid_constant__ CUtensorMap tm_a0,
+                             const __grid_constant__ CUtensorMap tm_b0,
+                             const __grid_constant__ CUtensorMap tm_sfa0,
+                             const __grid_constant__ CUtensorMap tm_sfb0,
+                             const __grid_constant__ CUtensorMap tm_d0,
+                             const __grid_constant__ CUtensorMap tm_a1,
+                             const __grid_constant__ CUtensorMap tm_b1,
+                             const __grid_constant__ CUtensorMap tm_sfa1,
+                             const __grid_constant__ CUtensorMap tm_sfb1,
+                             const __grid_constant__ CUtensorMap tm_d1,
+                             const __grid_constant__ GemmParams p) {
   using C = GemmCfg<CG, BN, BK>;
   constexpr int S = C::kStages;
   constexpr int NA = C::kNacc;
@@ -174,7 +253,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
   const bool leader = (rank == 0);
   const int cluster_id = blockIdx.x / CG;
   const int num_clusters = gridDim.x / CG;
-  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int nunits = unit_count(p, cluster_id, num_clusters);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -190,11 +269,18 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tm_a);
-    prefetch_tmap(&tm_b);
-    prefetch_tmap(&tm_sfa);
-    prefetch_tmap(&tm_sfb);
-    prefetch_tmap(&tm_d);
+    prefetch_tmap(&tm_a0);
+    prefetch_tmap(&tm_b0);
+    prefetch_tmap(&tm_sfa0);
+    prefetch_tmap(&tm_sfb0);
+    prefetch_tmap(&tm_d0);
+    if (p.nprob > 1) {
+      prefetch_tmap(&tm_a1);
+      prefetch_tmap(&tm_b1);
+      prefetch_tmap(&tm_sfa1);
+      prefetch_tmap(&tm_sfb1);
+      prefetch_tmap(&tm_d1);
+    }
   }
   if (warp == 1) {
     tmem_alloc<CG>(tmem_slot, 512);
@@ -215,11 +301,19 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     int sfc = 0;  // scale chunks loaded so far (ring position)
     uint32_t issued_mask = 0, issued_phase = 0;
     bool ok = true;
-    for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
-      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    for (int ui = 0; ui < nunits && ok; ++ui) {
+      const int u = unit_at(p, cluster_id, num_clusters, ui);
+      const int pr = u >= p.tiles0 ? 1 : 0;
+      const int tile = u - (pr ? p.tiles0 : 0);
+      const GemmProblem& P = p.prob[pr];
+      const CUtensorMap* tm_a = pr ? &tm_a1 : &tm_a0;
+      const CUtensorMap* tm_b = pr ? &tm_b1 : &tm_b0;
+      const CUtensorMap* tm_sfa = pr ? &tm_sfa1 : &tm_sfa0;
+      const CUtensorMap* tm_sfb = pr ? &tm_sfb1 : &tm_sfb0;
+      const int tm = tile % P.tiles_m, tn = tile / P.tiles_m;
       const int a_row = tm * C::kBM + 128 * (int)rank;
       const int b_row = tn * BN + C::kBNC * (int)rank;
-      for (int kb = 0; kb < p.kblocks; ++kb) {
+      for (int kb = 0; kb < P.kblocks; ++kb) {
         if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
         const bool sf = (kb % C::kStagesPerSf) == 0;
         const int slot = sfc % R;
@@ -228,13 +322,13 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
           if (leader)
             mbar_arrive_expect_tx(&full[stage], C::kTxPerStage + (sf ? C::kTxPerSf : 0u));
           const uint32_t bar = leader_addr<CG>(&full[stage]);
-          tma_load_2d<CG>(smem + C::kOffA + stage * C::kABytes, &tm_a, kb * BK, a_row, bar);
-          tma_load_2d<CG>(smem + C::kOffB + stage * C::kBBytes, &tm_b, kb * BK, b_row, bar);
+          tma_load_2d<CG>(smem + C::kOffA + stage * C::kABytes, tm_a, kb * BK, a_row, bar);
+          tma_load_2d<CG>(smem + C::kOffB + stage * C::kBBytes, tm_b, kb * BK, b_row, bar);
           if (sf) {
             uint8_t* sfbuf = smem + C::kOffSf + slot * C::kSfSlotBytes;
             const int chunk = kb / C::kStagesPerSf;
-            tma_load_3d<CG>(sfbuf, &tm_sfa, 0, chunk, a_row >> 7, bar);
-            tma_load_3d<CG>(sfbuf + C::kSfaBytes, &tm_sfb, 0, chunk, (tn * BN) >> 7, bar);
+            tma_load_3d<CG>(sfbuf, tm_sfa, 0, chunk, a_row >> 7, bar);
+            tma_load_3d<CG>(sfbuf + C::kSfaBytes, tm_sfb, 0, chunk, (tn * BN) >> 7, bar);
           }
         }
         if (sf) ++sfc;
@@ -261,7 +355,9 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       int sfc = 0;  // scale chunks copied to TMEM so far
       const uint64_t adesc0 = desc_kmajor<BK>(smem_u32(smem + C::kOffA));
       const uint64_t bdesc0 = desc_kmajor<BK>(smem_u32(smem + C::kOffB));
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++it) {
+      for (int ui = 0; ui < nunits && ok; ++ui, ++it) {
+        const int u = unit_at(p, cluster_id, num_clusters, ui);
+        const int kblocks = p.prob[u >= p.tiles0 ? 1 : 0].kblocks;
         const int acc = it % NA;
         const uint32_t acc_phase = (it / NA) & 1;
         if (!mbar_wait_warp(&acce[acc], acc_phase ^ 1, abort_flag)) break;
@@ -273,7 +369,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
         tc_fence_after();
         const uint32_t t_acc = tmem + acc * BN;
         const uint32_t t_sfreg = tmem + (C::kSfInTail ? (uint32_t)((acc ^ 1) * BN + BN - 32) : C::kSfCol);
-        for (int kb = 0; kb < p.kblocks; ++kb) {
+        for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_warp(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           if ((kb % C::kStagesPerSf) == 0) {
@@ -322,8 +418,12 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     uint8_t* ebuf = smem + C::kOffEpi + (warp - 2) * C::kEpiBufs * C::kEpiChunkBytes;
     int ebufc = 0;  // chunks staged so far (staging buffer ring position)
     int it = 0;
-    for (int tile = cluster_id; tile < num_tiles; tile += num_clusters, ++it) {
-      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+    for (int ui = 0; ui < nunits; ++ui, ++it) {
+      const int u = unit_at(p, cluster_id, num_clusters, ui);
+      const int pr = u >= p.tiles0 ? 1 : 0;
+      const int tile = u - (pr ? p.tiles0 : 0);
+      const GemmProblem& P = p.prob[pr];
+      const int tm = tile % P.tiles_m, tn = tile / P.tiles_m;
       const int acc = it % NA;
       const uint32_t acc_phase = (it / NA) & 1;
       if (!mbar_wait(&accf[acc], acc_phase, abort_flag)) break;
@@ -357,48 +457,12 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader<CG>(&acce[acc]);
-      // rows through this warp's staging buffers: lane = row, 64 bytes (32 BF16
-      // or 16 FP32 columns) per chunk; one TMA store (or reduce-add) per chunk
-      // writes 32 rows x 64 B
-      constexpr int kCC = (OUT == kOutBf16) ? 32 : 16;  // columns per chunk
       const int row0 = tm * C::kBM + 128 * (int)rank + sp * 32;
       const int gcol = tn * BN + half * C::kEpiCols;
-      if (row0 < p.rows_a) {
-#pragma unroll
-        for (int c = 0; c < C::kEpiCols / kCC; ++c) {
-          if (gcol + c * kCC < p.rows_b) {
-            uint8_t* buf = ebuf + (ebufc % C::kEpiBufs) * C::kEpiChunkBytes;
-            if (lane == 0) bulk_wait_group_read<C::kEpiBufs - 1>();
-            __syncwarp();
-            uint32_t pk[16];
-            if (OUT == kOutBf16) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[c * 32 + 2 * e]),
-                                                         __uint_as_float(r[c * 32 + 2 * e + 1]));
-                pk[e] = *reinterpret_cast<uint32_t*>(&h);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) pk[e] = r[c * 16 + e];
-            }
-            uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              if (OUT == kOutF32Add)
-                tma_reduce_add_2d(&tm_d, buf, gcol + c * kCC, row0);
-              else
-                tma_store_2d(&tm_d, buf, gcol + c * kCC, row0);
-              bulk_commit_group();
-            }
-            ++ebufc;
-          }
-        }
-      }
+      if (pr == 0)
+        epilogue_store<C, OUT0>(r, &tm_d0, ebuf, ebufc, lane, row0, gcol, P.rows_a, P.rows_b);
+      else
+        epilogue_store<C, OUT1>(r, &tm_d1, ebuf, ebufc, lane, row0, gcol, P.rows_a, P.rows_b);
     }
     // the staging buffers must stay valid until the stores have read them
     if (lane == 0) bulk_wait_group<0>();

@@ -9,9 +9,13 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <functional>
 #include <mutex>
+#include <queue>
+#include <vector>
 
 #include "../../include/puro_fp8.h"
 #include "common.cuh"
@@ -171,33 +175,74 @@ struct GemmArgs {
   int out;                          // puro::GemmOut
 };
 
+// Tensor maps of one GEMM: operands, their scales and the output.
 template <int CG, int BN, int BK, int OUT>
-int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
+int make_gemm_maps(const GemmArgs& g, CUtensorMap* m) {
   using C = puro::GemmCfg<CG, BN, BK>;
-  CUtensorMap ma, mb, msa, msb;
   const int64_t kb = (g.k + 127) / 128;
   int st;
   const CUtensorMapSwizzle sw = BK == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if ((st = make_map_u8(&ma, g.a, g.k, g.rows_a, g.lda, BK, 128, sw)) != PURO_OK) return st;
-  if ((st = make_map_u8(&mb, g.b, g.k, g.rows_b, g.ldb, BK, C::kBNC, sw)) != PURO_OK) return st;
-  if ((st = make_map_scales(&msa, g.sfa, g.rows_a, kb, 1)) != PURO_OK) return st;
-  if ((st = make_map_scales(&msb, g.sfb, g.rows_b, kb, C::kNB)) != PURO_OK) return st;
+  if ((st = make_map_u8(&m[0], g.a, g.k, g.rows_a, g.lda, BK, 128, sw)) != PURO_OK) return st;
+  if ((st = make_map_u8(&m[1], g.b, g.k, g.rows_b, g.ldb, BK, C::kBNC, sw)) != PURO_OK) return st;
+  if ((st = make_map_scales(&m[2], g.sfa, g.rows_a, kb, 1)) != PURO_OK) return st;
+  if ((st = make_map_scales(&m[3], g.sfb, g.rows_b, kb, C::kNB)) != PURO_OK) return st;
   // output [rows_a, rows_b], row stride ldd elements; store boxes of 32 rows
   // x 64 bytes (32 BF16 or 16 FP32 columns)
-  CUtensorMap md;
-  {
-    const bool f32 = OUT != puro::kOutBf16;
-    cuuint64_t dims[2] = {(cuuint64_t)g.rows_b, (cuuint64_t)g.rows_a};
-    cuuint64_t strides[1] = {(cuuint64_t)g.ldd * (f32 ? 4 : 2)};
-    cuuint32_t box[2] = {f32 ? 16u : 32u, 32};
-    cuuint32_t estr[2] = {1, 1};
-    if (g_encode(&md, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                 g.d, dims, strides, box, estr,
-                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return PURO_ERR_CUDA;
+  const bool f32 = OUT != puro::kOutBf16;
+  cuuint64_t dims[2] = {(cuuint64_t)g.rows_b, (cuuint64_t)g.rows_a};
+  cuuint64_t strides[1] = {(cuuint64_t)g.ldd * (f32 ? 4 : 2)};
+  cuuint32_t box[2] = {f32 ? 16u : 32u, 32};
+  cuuint32_t estr[2] = {1, 1};
+  if (g_encode(&m[4], f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.d,
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return PURO_ERR_CUDA;
+  return PURO_OK;
+}
+
+// Longest-processing-time-first assignment of the two problems' tiles to
+// `clusters` clusters: tiles in order of decreasing cost (K blocks plus a
+// fixed per-tile share for the epilogue), each to the least-loaded cluster;
+// every cluster runs its tiles in the order they were assigned.
+void make_schedule(puro::GemmParams& p, int clusters) {
+  const int units = p.units;
+  std::vector<int> order(units);
+  for (int u = 0; u < units; ++u) order[u] = u;
+  auto cost = [&](int u) { return p.prob[u >= p.tiles0 ? 1 : 0].kblocks + 2; };
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return cost(x) > cost(y); });
+  using Slot = std::pair<int64_t, int>;  // (load, cluster), least load first, then lowest index
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int c = 0; c < clusters; ++c) heap.push({0, c});
+  std::vector<std::vector<int>> lists(clusters);
+  for (int u : order) {
+    Slot s = heap.top();
+    heap.pop();
+    lists[s.second].push_back(u);
+    heap.push({s.first + cost(u), s.second});
   }
-  auto kern = puro::gemm_block_scaled_kernel<CG, BN, BK, OUT>;
+  int off = 0;
+  for (int c = 0; c < clusters; ++c) {
+    p.sched_off[c] = (uint16_t)off;
+    for (int u : lists[c]) p.sched_unit[off++] = (uint16_t)u;
+  }
+  p.sched_off[clusters] = (uint16_t)off;
+  p.sched = 1;
+}
+
+// One launch of the GEMM kernel over one problem (g1 == nullptr) or two
+// independent problems that share the launch.
+template <int CG, int BN, int BK, int OUT0, int OUT1>
+int launch_gemm_cfg(const GemmArgs& g0, const GemmArgs* g1, DeviceInfo* dev, cudaStream_t stream) {
+  using C = puro::GemmCfg<CG, BN, BK>;
+  CUtensorMap m0[5], m1[5];
+  int st;
+  if ((st = make_gemm_maps<CG, BN, BK, OUT0>(g0, m0)) != PURO_OK) return st;
+  if (g1) {
+    if ((st = make_gemm_maps<CG, BN, BK, OUT1>(*g1, m1)) != PURO_OK) return st;
+  } else {
+    memcpy(m1, m0, sizeof(m0));  // unused by a one-problem launch
+  }
+  auto kern = puro::gemm_block_scaled_kernel<CG, BN, BK, OUT0, OUT1>;
   static int max_clusters[kMaxDevices] = {};
   int dev_id = 0;
   cudaGetDevice(&dev_id);
@@ -221,19 +266,31 @@ int launch_gemm_cfg(const GemmArgs& g, DeviceInfo* dev, cudaStream_t stream) {
     int n = 0;
     cfg.gridDim = dim3(CG * (dev->sms / CG));
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = dev->sms / CG;
-    max_clusters[dev_id] = n;
+    max_clusters[dev_id] = n < puro::kMaxSchedClusters ? n : puro::kMaxSchedClusters;
   }
-  puro::GemmParams p;
-  p.rows_a = (int32_t)g.rows_a;
-  p.rows_b = (int32_t)g.rows_b;
-  p.kblocks = (int32_t)((g.k + BK - 1) / BK);
-  p.tiles_m = (int32_t)((g.rows_a + C::kBM - 1) / C::kBM);
-  p.tiles_n = (int32_t)((g.rows_b + BN - 1) / BN);
-  const int tiles = p.tiles_m * p.tiles_n;
-  const int clusters = tiles < max_clusters[dev_id] ? tiles : max_clusters[dev_id];
+  static thread_local puro::GemmParams p;  // ~4.5 KB: kept off the stack
+  memset(&p, 0, sizeof(p));
+  const GemmArgs* gs[2] = {&g0, g1};
+  p.nprob = g1 ? 2 : 1;
+  for (int i = 0; i < p.nprob; ++i) {
+    const GemmArgs& g = *gs[i];
+    p.prob[i].rows_a = (int32_t)g.rows_a;
+    p.prob[i].rows_b = (int32_t)g.rows_b;
+    p.prob[i].kblocks = (int32_t)((g.k + BK - 1) / BK);
+    p.prob[i].tiles_m = (int32_t)((g.rows_a + C::kBM - 1) / C::kBM);
+    p.prob[i].tiles_n = (int32_t)((g.rows_b + BN - 1) / BN);
+  }
+  const int64_t t0 = (int64_t)p.prob[0].tiles_m * p.prob[0].tiles_n;
+  const int64_t t1 = g1 ? (int64_t)p.prob[1].tiles_m * p.prob[1].tiles_n : 0;
+  p.tiles0 = (int32_t)t0;
+  p.units = (int32_t)(t0 + t1);
+  const int clusters = p.units < max_clusters[dev_id] ? p.units : max_clusters[dev_id];
+  if (g1 && p.units <= puro::kMaxSchedUnits) make_schedule(p, clusters);
   cfg.gridDim = dim3(CG * clusters);
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, md, p) != cudaSuccess) return PURO_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, m0[0], m0[1], m0[2], m0[3], m0[4], m1[0], m1[1], m1[2], m1[3],
+                         m1[4], p) != cudaSuccess)
+    return PURO_ERR_CUDA;
   return launch_status();
 }
 
@@ -252,13 +309,43 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream) {
       return PURO_ERR_CUDA;
     return PURO_OK;
   }
+  constexpr int CG = PURO_GEMM_CG, BN = PURO_GEMM_BN, BK = PURO_GEMM_BK;
   switch (g.out) {
     case puro::kOutBf16:
-      return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN, PURO_GEMM_BK, puro::kOutBf16>(g, dev, stream);
+      return launch_gemm_cfg<CG, BN, BK, puro::kOutBf16, puro::kOutBf16>(g, nullptr, dev, stream);
     case puro::kOutF32:
-      return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN, PURO_GEMM_BK, puro::kOutF32>(g, dev, stream);
+      return launch_gemm_cfg<CG, BN, BK, puro::kOutF32, puro::kOutF32>(g, nullptr, dev, stream);
     case puro::kOutF32Add:
-      return launch_gemm_cfg<PURO_GEMM_CG, PURO_GEMM_BN, PURO_GEMM_BK, puro::kOutF32Add>(g, dev, stream);
+      return launch_gemm_cfg<CG, BN, BK, puro::kOutF32Add, puro::kOutF32Add>(g, nullptr, dev, stream);
+    default:
+      return PURO_ERR_LAYOUT;
+  }
+}
+
+// Two independent GEMMs in one launch: g0 with a BF16 output (the data
+// gradient) and g1 with any output kind (the weight gradient).  A problem
+// that is empty, or has an empty reduction, is run on its own.
+int launch_gemm_pair(const GemmArgs& g0, const GemmArgs& g1, cudaStream_t stream) {
+  const bool e0 = g0.rows_a == 0 || g0.rows_b == 0 || g0.k == 0;
+  const bool e1 = g1.rows_a == 0 || g1.rows_b == 0 || g1.k == 0;
+  if (e0 || e1) {
+    int st = launch_gemm(g0, stream);
+    if (st != PURO_OK) return st;
+    return launch_gemm(g1, stream);
+  }
+  DeviceInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != PURO_OK) return st;
+  if ((st = get_encoder()) != PURO_OK) return st;
+  constexpr int CG = PURO_GEMM_CG, BN = PURO_GEMM_BN, BK = PURO_GEMM_BK;
+  if (g0.out != puro::kOutBf16) return PURO_ERR_LAYOUT;
+  switch (g1.out) {
+    case puro::kOutBf16:
+      return launch_gemm_cfg<CG, BN, BK, puro::kOutBf16, puro::kOutBf16>(g0, &g1, dev, stream);
+    case puro::kOutF32:
+      return launch_gemm_cfg<CG, BN, BK, puro::kOutBf16, puro::kOutF32>(g0, &g1, dev, stream);
+    case puro::kOutF32Add:
+      return launch_gemm_cfg<CG, BN, BK, puro::kOutBf16, puro::kOutF32Add>(g0, &g1, dev, stream);
     default:
       return PURO_ERR_LAYOUT;
   }
@@ -276,6 +363,47 @@ int check_mat(const void* p, int64_t ld, int64_t min_ld, int64_t elem_bytes) {
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
 
 }  // namespace
+
+// Argument checks and GEMM mapping of the gradient GEMMs.  They return
+// PURO_OK with *g filled in, kNothingToDo when the output is empty, or an
+// error status; nothing is launched.
+constexpr int kNothingToDo = 1;
+
+int dgrad_args(const void* qdy, int64_t ld_qdy, const void* sdy, const void* qwt, int64_t ld_qwt,
+               const void* sw_bwd, void* dx, int64_t ld_dx, int64_t m, int64_t n, int64_t k,
+               GemmArgs* g) {
+  if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
+  if (n % 128 || k % 128) return PURO_ERR_SHAPE;
+  if (m == 0 || k == 0) return kNothingToDo;
+  int r;
+  if ((r = check_mat(dx, ld_dx, k, 2)) != PURO_OK) return r;
+  if (n > 0) {
+    if ((r = check_mat(qdy, ld_qdy, n, 1)) != PURO_OK) return r;
+    if ((r = check_mat(qwt, ld_qwt, n, 1)) != PURO_OK) return r;
+    if (!sdy || !sw_bwd) return PURO_ERR_NULL;
+    if (!aligned16(sdy) || !aligned16(sw_bwd)) return PURO_ERR_ALIGN;
+  }
+  *g = GemmArgs{qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, k, n, puro::kOutBf16};
+  return PURO_OK;
+}
+
+int wgrad_args(const void* qdyt, int64_t ld_qdyt, const void* sdyt, const void* qxt, int64_t ld_qxt,
+               const void* sxt, void* dw, int64_t ld_dw, int64_t m, int64_t n, int64_t k, int out,
+               GemmArgs* g) {
+  if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
+  if (n % 128 || k % 128) return PURO_ERR_SHAPE;
+  if (n == 0 || k == 0) return kNothingToDo;
+  int r;
+  if ((r = check_mat(dw, ld_dw, k, out == puro::kOutBf16 ? 2 : 4)) != PURO_OK) return r;
+  if (m > 0) {
+    if ((r = check_mat(qdyt, ld_qdyt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
+    if ((r = check_mat(qxt, ld_qxt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
+    if (!sdyt || !sxt) return PURO_ERR_NULL;
+    if (!aligned16(sdyt) || !aligned16(sxt)) return PURO_ERR_ALIGN;
+  }
+  *g = GemmArgs{qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, n, k, m, out};
+  return PURO_OK;
+}
 
 extern "C" {
 
@@ -395,57 +523,49 @@ int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx, const voi
 int puro_fp8_gemm_dgrad(const void* qdy, int64_t ld_qdy, const void* sdy, const void* qwt,
                         int64_t ld_qwt, const void* sw_bwd, void* dx, int64_t ld_dx, int64_t m,
                         int64_t n, int64_t k, void* stream) {
-  if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
-  if (n % 128 || k % 128) return PURO_ERR_SHAPE;
-  if (m == 0 || k == 0) return PURO_OK;
-  int r;
-  if ((r = check_mat(dx, ld_dx, k, 2)) != PURO_OK) return r;
-  if (n > 0) {
-    if ((r = check_mat(qdy, ld_qdy, n, 1)) != PURO_OK) return r;
-    if ((r = check_mat(qwt, ld_qwt, n, 1)) != PURO_OK) return r;
-    if (!sdy || !sw_bwd) return PURO_ERR_NULL;
-    if (!aligned16(sdy) || !aligned16(sw_bwd)) return PURO_ERR_ALIGN;
-  }
-  GemmArgs g{qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, k, n, puro::kOutBf16};
+  GemmArgs g;
+  const int r = dgrad_args(qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, n, k, &g);
+  if (r != PURO_OK) return r == kNothingToDo ? PURO_OK : r;
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
 int puro_fp8_gemm_wgrad(const void* qdyt, int64_t ld_qdyt, const void* sdyt, const void* qxt,
                         int64_t ld_qxt, const void* sxt, void* dw, int64_t ld_dw, int64_t m,
                         int64_t n, int64_t k, void* stream) {
-  if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
-  if (n % 128 || k % 128) return PURO_ERR_SHAPE;
-  if (n == 0 || k == 0) return PURO_OK;
-  int r;
-  if ((r = check_mat(dw, ld_dw, k, 2)) != PURO_OK) return r;
-  if (m > 0) {
-    if ((r = check_mat(qdyt, ld_qdyt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
-    if ((r = check_mat(qxt, ld_qxt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
-    if (!sdyt || !sxt) return PURO_ERR_NULL;
-    if (!aligned16(sdyt) || !aligned16(sxt)) return PURO_ERR_ALIGN;
-  }
-  GemmArgs g{qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, n, k, m, puro::kOutBf16};
+  GemmArgs g;
+  const int r = wgrad_args(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k, puro::kOutBf16, &g);
+  if (r != PURO_OK) return r == kNothingToDo ? PURO_OK : r;
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
 }
 
 int puro_fp8_gemm_wgrad_f32(const void* qdyt, int64_t ld_qdyt, const void* sdyt, const void* qxt,
                             int64_t ld_qxt, const void* sxt, void* dw, int64_t ld_dw, int64_t m,
                             int64_t n, int64_t k, int accumulate, void* stream) {
-  if (m < 0 || n < 0 || k < 0 || m >= kMaxDim || n >= kMaxDim || k >= kMaxDim) return PURO_ERR_SHAPE;
-  if (n % 128 || k % 128) return PURO_ERR_SHAPE;
   if (accumulate != 0 && accumulate != 1) return PURO_ERR_LAYOUT;
-  if (n == 0 || k == 0) return PURO_OK;
-  int r;
-  if ((r = check_mat(dw, ld_dw, k, 4)) != PURO_OK) return r;
-  if (m > 0) {
-    if ((r = check_mat(qdyt, ld_qdyt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
-    if ((r = check_mat(qxt, ld_qxt, (m + 15) / 16 * 16, 1)) != PURO_OK) return r;
-    if (!sdyt || !sxt) return PURO_ERR_NULL;
-    if (!aligned16(sdyt) || !aligned16(sxt)) return PURO_ERR_ALIGN;
-  }
-  GemmArgs g{qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, n, k, m,
-             accumulate ? puro::kOutF32Add : puro::kOutF32};
+  GemmArgs g;
+  const int r = wgrad_args(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k,
+                           accumulate ? puro::kOutF32Add : puro::kOutF32, &g);
+  if (r != PURO_OK) return r == kNothingToDo ? PURO_OK : r;
   return launch_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+int puro_fp8_gemm_dgrad_wgrad(const void* qdy, int64_t ld_qdy, const void* sdy, const void* qwt,
+                              int64_t ld_qwt, const void* sw_bwd, void* dx, int64_t ld_dx,
+                              const void* qdyt, int64_t ld_qdyt, const void* sdyt, const void* qxt,
+                              int64_t ld_qxt, const void* sxt, void* dw, int64_t ld_dw, int64_t m,
+                              int64_t n, int64_t k, int dw_kind, void* stream) {
+  if (dw_kind < PURO_DW_BF16 || dw_kind > PURO_DW_F32_ACCUMULATE) return PURO_ERR_LAYOUT;
+  const int out = dw_kind == PURO_DW_BF16 ? puro::kOutBf16
+                  : dw_kind == PURO_DW_F32 ? puro::kOutF32 : puro::kOutF32Add;
+  GemmArgs gd, gw;
+  const int rd = dgrad_args(qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx, m, n, k, &gd);
+  if (rd != PURO_OK && rd != kNothingToDo) return rd;
+  const int rw = wgrad_args(qdyt, ld_qdyt, sdyt, qxt, ld_qxt, sxt, dw, ld_dw, m, n, k, out, &gw);
+  if (rw != PURO_OK && rw != kNothingToDo) return rw;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (rd == kNothingToDo) return rw == kNothingToDo ? PURO_OK : launch_gemm(gw, s);
+  if (rw == kNothingToDo) return launch_gemm(gd, s);
+  return launch_gemm_pair(gd, gw, s);
 }
 
 int puro_fp8_device_status(void* stream) {

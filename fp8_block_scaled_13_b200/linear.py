@@ -182,6 +182,42 @@ def gemm_wgrad(dyq: QuantAct, xq: QuantAct, out: torch.Tensor | None = None,
     return out
 
 
+def gemm_dgrad_wgrad(dyq: QuantAct, wq: QuantWeight, xq: QuantAct, dx: torch.Tensor | None = None,
+                     dw: torch.Tensor | None = None, accumulate: bool = False):
+    """dX = dY W and dW = dY^T X in one launch (tiles of both spread over the
+    GPU together); results identical to gemm_dgrad and gemm_wgrad.  `dw` BF16
+    (default) or FP32; accumulate=True adds into an FP32 `dw`.  Returns (dx, dw)."""
+    m, n, k = dyq.rows, dyq.cols, wq.k
+    if wq.n != n or xq.rows != m or xq.cols != k:
+        raise ValueError("shapes of dY, W and X do not agree")
+    if wq.qt is None:
+        raise ValueError("the weight was quantized without its transposed copy")
+    dev = dyq.q.device
+    if dx is None:
+        dx = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
+    if dw is None:
+        if accumulate:
+            raise ValueError("accumulate=True needs the FP32 buffer to add into")
+        dw = torch.empty((n, k), dtype=torch.bfloat16, device=dev)
+    if tuple(dw.shape) != (n, k) or dw.stride(1) != 1 or tuple(dx.shape) != (m, k) or dx.stride(1) != 1:
+        raise ValueError("dx must be row-major [m, k] and dw row-major [n, k]")
+    if dw.dtype == torch.float32:
+        kind = _lib.PURO_DW_F32_ACCUMULATE if accumulate else _lib.PURO_DW_F32
+    elif dw.dtype == torch.bfloat16 and not accumulate:
+        kind = _lib.PURO_DW_BF16
+    else:
+        raise ValueError("dw must be BF16, or FP32 (required for accumulate=True)")
+    st = _lib.puro_fp8_gemm_dgrad_wgrad(
+        dyq.q.data_ptr(), dyq.q.stride(0), dyq.s.data_ptr(),
+        wq.qt.data_ptr(), wq.qt.stride(0), wq.s_bwd.data_ptr(),
+        dx.data_ptr(), dx.stride(0),
+        dyq.qt.data_ptr(), dyq.qt.stride(0), dyq.st.data_ptr(),
+        xq.qt.data_ptr(), xq.qt.stride(0), xq.st.data_ptr(),
+        dw.data_ptr(), dw.stride(0), m, n, k, kind, _stream())
+    _check(st, "puro_fp8_gemm_dgrad_wgrad")
+    return dx, dw
+
+
 def device_status() -> int:
     """Synchronize the current stream and return/clear the device error word."""
     return _lib.puro_fp8_device_status(_stream())
@@ -201,7 +237,6 @@ def linear_backward(dy: torch.Tensor, xq: QuantAct, wq: QuantWeight,
     With `main_grad` (FP32 [n, k]) the weight gradient is added into it
     (gradient accumulation across micro-batches) and returned as dw."""
     dyq = quant_act(dy, "both")
-    dx = gemm_dgrad(dyq, wq)
     if main_grad is not None:
-        return dx, gemm_wgrad(dyq, xq, out=main_grad, accumulate=True)
-    return dx, gemm_wgrad(dyq, xq)
+        return gemm_dgrad_wgrad(dyq, wq, xq, dw=main_grad, accumulate=True)
+    return gemm_dgrad_wgrad(dyq, wq, xq)

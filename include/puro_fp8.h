@@ -194,6 +194,36 @@ PURO_API int puro_fp8_gemm_wgrad_f32(const void* qdyt, int64_t ld_qdyt, const vo
                                      void* dw, int64_t ld_dw, int64_t m, int64_t n, int64_t k,
                                      int accumulate, void* stream);
 
+/* Output kinds of the weight gradient in puro_fp8_gemm_dgrad_wgrad. */
+enum {
+  PURO_DW_BF16 = 0,            /* dW = dY^T X, BF16 (as puro_fp8_gemm_wgrad)               */
+  PURO_DW_F32 = 1,             /* dW = dY^T X, FP32 (as puro_fp8_gemm_wgrad_f32, acc. 0)   */
+  PURO_DW_F32_ACCUMULATE = 2   /* dW += dY^T X, FP32 (as puro_fp8_gemm_wgrad_f32, acc. 1)  */
+};
+
+/*
+ * puro_fp8_gemm_dgrad_wgrad -- the two backward GEMMs of one linear layer in
+ * one launch: dX = dY W (arguments and result exactly as puro_fp8_gemm_dgrad)
+ * and dW = dY^T X (as puro_fp8_gemm_wgrad, or the FP32 forms, by dw_kind).
+ * The two are independent given the quantized dY, X and W.  Sharing the launch
+ * only changes which SM computes which output tile: the tiles of both are
+ * assigned to the clusters longest-first (by K blocks) to the least-loaded
+ * cluster, so that neither GEMM leaves most of the GPU idle in a last,
+ * partly-filled wave of tiles.  Every output element is computed exactly as in
+ * the separate calls (bit-identical results).
+ * m, n, k: tokens, layer outputs, layer inputs (dY [m, n], X [m, k], W [n, k]).
+ * Errors as the separate calls; dw_kind outside PURO_DW_* -> PURO_ERR_LAYOUT.
+ * If either product is empty the other one runs on its own.
+ */
+PURO_API int puro_fp8_gemm_dgrad_wgrad(const void* qdy, int64_t ld_qdy, const void* sdy,
+                                       const void* qwt, int64_t ld_qwt, const void* sw_bwd,
+                                       void* dx, int64_t ld_dx,
+                                       const void* qdyt, int64_t ld_qdyt, const void* sdyt,
+                                       const void* qxt, int64_t ld_qxt, const void* sxt,
+                                       void* dw, int64_t ld_dw,
+                                       int64_t m, int64_t n, int64_t k, int dw_kind,
+                                       void* stream);
+
 /*
  * puro_fp8_device_status -- synchronizes `stream`, then returns and clears the
  * library's device error word for the current device: PURO_OK, or

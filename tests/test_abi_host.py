@@ -125,11 +125,37 @@ def test_wgrad_f32_argument_errors(lib, args, code):
     assert lib.puro_fp8_gemm_wgrad_f32(*args, None) == code
 
 
+def _dw_args(**over):
+    # dgrad (qdy, ld_qdy, sdy, qwt, ld_qwt, sw_bwd, dx, ld_dx), wgrad (qdyt, ld_qdyt, sdyt, qxt,
+    # ld_qxt, sxt, dw, ld_dw), m, n, k, dw_kind
+    a = dict(qdy=A, ld_qdy=256, sdy=A, qwt=A, ld_qwt=256, sw=A, dx=A, ld_dx=256,
+             qdyt=A, ld_qdyt=64, sdyt=A, qxt=A, ld_qxt=64, sxt=A, dw=A, ld_dw=256,
+             m=64, n=256, k=256, kind=0)
+    a.update(over)
+    return tuple(a.values())
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(kind=3), -4),                 # unknown dW kind
+    (dict(kind=-1), -4),
+    (dict(n=200), -3),                  # n % 128
+    (dict(sw=None), -1),                # the dgrad part's checks
+    (dict(ld_dx=100), -3),
+    (dict(sxt=None), -1),               # the wgrad part's checks
+    (dict(ld_dw=258, kind=1), -2),      # FP32 dW row stride not a multiple of 16 bytes
+    (dict(ld_qdyt=48), -3),
+])
+def test_dgrad_wgrad_argument_errors(lib, over, code):
+    assert lib.puro_fp8_gemm_dgrad_wgrad(*_dw_args(**over), None) == code
+
+
 def test_gemm_empty_is_noop(lib):
     assert lib.puro_fp8_gemm_fprop(None, 0, None, None, 0, None, None, 0, 0, 256, 256, None) == 0
     assert lib.puro_fp8_gemm_wgrad(None, 0, None, None, 0, None, None, 0, 64, 0, 256, None) == 0
     assert lib.puro_fp8_gemm_wgrad_f32(None, 0, None, None, 0, None, None, 0, 64, 0, 256, 1,
                                        None) == 0
+    # n == 0: both the data and the weight gradient are empty
+    assert lib.puro_fp8_gemm_dgrad_wgrad(*_dw_args(n=0, k=0), None) == 0
 
 
 @pytest.mark.parametrize("rows,groups,want", [

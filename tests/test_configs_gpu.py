@@ -81,6 +81,12 @@ def _check_layer(fp8, oracle_mod, L, seed):
     cols = _sample(n, N_ROWS, seed + 2)
     ref = oracle_mod.linear_wgrad(L.dy[:, cols].contiguous(), L.x)
     assert_gemm_close(dw[cols.tolist()], ref, oracle_mod, "%s wgrad" % L.name)
+    # both backward GEMMs in one launch: bit-identical to the separate calls
+    dx2, dw2 = fp8.gemm_dgrad_wgrad(dyq, wq, xq)
+    torch.cuda.synchronize()
+    assert torch.equal(dx2.view(torch.int16), dx.view(torch.int16))
+    assert torch.equal(dw2.view(torch.int16), dw.view(torch.int16))
+    del dx2, dw2
     # the FP32 gradient buffer path: accumulate into an initialised buffer
     init = torch.full((n, k), 0.25, dtype=torch.float32, device=dev)
     fp8.gemm_wgrad(dyq, xq, out=init, accumulate=True)

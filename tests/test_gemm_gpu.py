@@ -114,3 +114,34 @@ def test_output_strides(fp8, oracle_mod):
     torch.cuda.synchronize()
     assert torch.all(buf[:, :128] == -1) and torch.all(buf[:, 384:] == -1)
     assert_gemm_close(buf[:, 128:384], oracle_mod.linear_fprop(x, w), oracle_mod, "strided fprop")
+
+
+@pytest.mark.parametrize("m,n,k", [
+    (300, 384, 512),      # ragged tokens
+    (129, 256, 384),
+    (1000, 640, 768),     # tile counts and K differ between the two products
+    (128, 16384, 128),    # dgrad tiles exceed the schedule table: round-robin fallback
+])
+@pytest.mark.parametrize("kind", ["bf16", "f32", "f32_accumulate"])
+def test_dgrad_wgrad_launch_matches_separate_calls(fp8, m, n, k, kind):
+    """One launch for both backward GEMMs computes every element exactly as
+    the separate calls do (only the tile-to-SM assignment differs)."""
+    x, w, dy = _layer(m, n, k, 3 * m + n)
+    dev = torch.device("cuda")
+    xq = fp8.quant_act(x.to(dev), "colwise")
+    wq = fp8.quant_weight(w.to(dev), transpose=True)
+    dyq = fp8.quant_act(dy.to(dev), "both")
+    dx_ref = fp8.gemm_dgrad(dyq, wq)
+    if kind == "bf16":
+        dw_ref = fp8.gemm_wgrad(dyq, xq)
+        dx, dw = fp8.gemm_dgrad_wgrad(dyq, wq, xq)
+    else:
+        init = torch.randn(n, k, generator=torch.Generator().manual_seed(9)).to(dev)
+        acc = kind == "f32_accumulate"
+        dw_ref = fp8.gemm_wgrad(dyq, xq, out=init.clone(), accumulate=acc)
+        dx, dw = fp8.gemm_dgrad_wgrad(dyq, wq, xq, dw=init.clone(), accumulate=acc)
+    torch.cuda.synchronize()
+    assert fp8.device_status() == 0
+    assert torch.equal(dx.view(torch.int16), dx_ref.view(torch.int16))
+    assert torch.equal(dw.view(torch.int16 if kind == "bf16" else torch.int32),
+                       dw_ref.view(torch.int16 if kind == "bf16" else torch.int32))

@@ -36,7 +36,7 @@ M_TOKENS = 8192
 # dram__bytes_read.sum + dram__bytes_write.sum of one GEMM launch (fprop, QKV
 # layer) from the ncu capture summarised in profiles/; None until captured
 # for the current kernel.
-GEMM_TRAFFIC_BYTES = None  # recaptured after the scheduled-launch change (profiles/)
+GEMM_TRAFFIC_BYTES = 23327744 + 6664960  # QKV fprop launch, profiles/gemm_block_scaled_attn_proj_qkv_fprop.md
 
 
 def _peaks():
@@ -525,39 +525,83 @@ def run_e2e(wl, dev, K, warmup):
     """Same step through the public API with pinned host inputs/outputs: every
     step copies X, W, dY in, runs forward and backward (dW added into the FP32
     main grads), and copies Y, dX and the main grads back, all inside the
-    timed region."""
+    timed region.  The copies are pipelined across steps the way a training
+    loop would: step i+1's inputs go up on a copy stream while step i
+    computes, and step i's results come down on another while step i+1
+    computes (double-buffered device and host buffers, ordered by events)."""
     import torch
     import fp8_block_scaled_13_b200 as fp8
     from fp8_block_scaled_13_b200.dp import MainGrads
 
-    host_in = [(L.x.pin_memory(), L.w.pin_memory(), L.dy.pin_memory()) for L in wl.layers]
-    host_out = [(torch.empty((L.m, L.n), dtype=torch.bfloat16).pin_memory(),
-                 torch.empty((L.m, L.k), dtype=torch.bfloat16).pin_memory(),
-                 torch.empty((L.n, L.k), dtype=torch.float32).pin_memory()) for L in wl.layers]
-    grads = MainGrads([(L.n, L.k) for L in wl.layers], device=dev)
-    h2d = sum(t.numel() * t.element_size() for tup in host_in for t in tup)
-    d2h = sum(t.numel() * t.element_size() for tup in host_out for t in tup)
+    nbuf = 2
+    host_in = [[(L.x.pin_memory(), L.w.pin_memory(), L.dy.pin_memory()) for L in wl.layers]
+               for _ in range(nbuf)]
+    host_out = [[(torch.empty((L.m, L.n), dtype=torch.bfloat16).pin_memory(),
+                  torch.empty((L.m, L.k), dtype=torch.bfloat16).pin_memory(),
+                  torch.empty((L.n, L.k), dtype=torch.float32).pin_memory()) for L in wl.layers]
+                for _ in range(nbuf)]
+    dev_in = [[(torch.empty_like(x, device=dev), torch.empty_like(w, device=dev),
+                torch.empty_like(dy, device=dev)) for (x, w, dy) in host_in[0]] for _ in range(nbuf)]
+    results = [None] * nbuf   # device outputs (Y, dX) of the step that used buffer b
+    grads = [MainGrads([(L.n, L.k) for L in wl.layers], device=dev) for _ in range(nbuf)]
+    h2d = sum(t.numel() * t.element_size() for tup in host_in[0] for t in tup)
+    d2h = sum(t.numel() * t.element_size() for tup in host_out[0] for t in tup)
+    comp = torch.cuda.current_stream()
+    up = torch.cuda.Stream()
+    down = torch.cuda.Stream()
+    ev_up = [torch.cuda.Event() for _ in range(nbuf)]      # inputs of buffer b are on the device
+    ev_done = [torch.cuda.Event() for _ in range(nbuf)]    # compute on buffer b finished
+    ev_down = [torch.cuda.Event() for _ in range(nbuf)]    # results of buffer b are on the host
 
-    def one():
-        for li, ((hx, hw, hdy), (hy, hdx, hdw)) in enumerate(zip(host_in, host_out)):
-            x = hx.to(dev, non_blocking=True)
-            w = hw.to(dev, non_blocking=True)
-            dy = hdy.to(dev, non_blocking=True)
+    def upload(i):
+        b = i % nbuf
+        with torch.cuda.stream(up):
+            up.wait_event(ev_done[b])   # the previous use of these device inputs is over
+            for (hx, hw, hdy), (x, w, dy) in zip(host_in[b], dev_in[b]):
+                x.copy_(hx, non_blocking=True)
+                w.copy_(hw, non_blocking=True)
+                dy.copy_(hdy, non_blocking=True)
+            ev_up[b].record(up)
+
+    def compute(i):
+        b = i % nbuf
+        comp.wait_event(ev_up[b])
+        comp.wait_event(ev_down[b])   # the previous results of buffer b went down
+        outs = []
+        for li, (x, w, dy) in enumerate(dev_in[b]):
             y, xq, wq = fp8.linear_forward(x, w)
-            dx, dw = fp8.linear_backward(dy, xq, wq, main_grad=grads[li])
-            hy.copy_(y, non_blocking=True)
-            hdx.copy_(dx, non_blocking=True)
-            hdw.copy_(dw, non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+            dx, _ = fp8.linear_backward(dy, xq, wq, main_grad=grads[b][li])
+            y.record_stream(down)
+            dx.record_stream(down)
+            outs.append((y, dx))
+        results[b] = outs
+        ev_done[b].record(comp)
 
-    for _ in range(warmup):
-        one()
-    torch.cuda.synchronize()
+    def download(i):
+        b = i % nbuf
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[b])
+            for li, ((hy, hdx, hdw), (y, dx)) in enumerate(zip(host_out[b], results[b])):
+                hy.copy_(y, non_blocking=True)
+                hdx.copy_(dx, non_blocking=True)
+                hdw.copy_(grads[b][li], non_blocking=True)
+            ev_down[b].record(down)
+
+    def run(n):
+        upload(0)
+        for i in range(n):
+            if i + 1 < n:
+                upload(i + 1)
+            compute(i)
+            download(i)
+        torch.cuda.synchronize()
+
+    run(warmup)
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
     s.record()
-    for _ in range(K):
-        one()
+    run(K)
     e.record()
     torch.cuda.synchronize()
     return {"ms_per_step": s.elapsed_time(e) / K, "h2d": h2d, "d2h": d2h}

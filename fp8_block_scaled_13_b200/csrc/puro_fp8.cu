@@ -123,8 +123,8 @@ int launch_status() {
 
 // ------------------------------------------------------------------ quant
 
-template <bool ROW, bool COL, bool BLOCK>
-int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, int sms,
+template <bool ROW, bool COL, bool BLOCK, bool RSHFL>
+int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, int sms,
                  cudaStream_t stream) {
   int st = get_encoder();
   if (st != PURO_OK) return st;
@@ -138,7 +138,7 @@ int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, int sm
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return PURO_ERR_CUDA;
-  auto kern = puro::quant_kernel<ROW, COL, BLOCK>;
+  auto kern = puro::quant_kernel<ROW, COL, BLOCK, RSHFL>;
   constexpr uint32_t smem = puro::quant_smem_bytes();
   static bool attr_done[kMaxDevices] = {};
   int dev_id = 0;
@@ -161,6 +161,16 @@ int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, int sm
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, m, p) != cudaSuccess) return PURO_ERR_CUDA;
   return launch_status();
+}
+
+// Row scales by shuffles when each CTA has few tiles (measured faster up to
+// about 8 tiles per CTA; the redundant per-thread form wins on long streams).
+template <bool ROW, bool COL, bool BLOCK>
+int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, int sms,
+                 cudaStream_t stream) {
+  if (ROW && !BLOCK && p.tiles <= 8 * 2 * (int64_t)sms)
+    return launch_quant_cfg<ROW, COL, BLOCK, true>(x, ld_x, p, sms, stream);
+  return launch_quant_cfg<ROW, COL, BLOCK, false>(x, ld_x, p, sms, stream);
 }
 
 // ------------------------------------------------------------------ gemm

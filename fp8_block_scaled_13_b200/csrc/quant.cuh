@@ -133,7 +133,12 @@ __device__ __forceinline__ uint4 lds_v4(const uint8_t* p) {
   return *reinterpret_cast<const uint4*>(p);
 }
 
-template <bool ROW, bool COL, bool BLOCK>
+// RSHFL selects how the row scales reach the threads (ROW without BLOCK):
+// one thread per row derives the exponent and the 16 threads of the row read
+// it with shuffles (fewer ALU instructions: faster when each CTA has only a
+// few tiles), or all 16 derive it themselves (no cross-lane latency on the
+// encode path: faster on long tile streams).  Both give identical results.
+template <bool ROW, bool COL, bool BLOCK, bool RSHFL>
 __global__ void __launch_bounds__(kQThreads, 2)
     quant_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantParams p) {
   constexpr uint32_t kMag = 0x7FFF7FFFu;
@@ -144,8 +149,8 @@ __global__ void __launch_bounds__(kQThreads, 2)
   uint8_t* tiles = smem;                                    // kQStages x 32 KB
   uint8_t* qt_s = smem + kQStages * kQTileBytes;            // 16 KB transposed codes
   uint32_t* col_part = reinterpret_cast<uint32_t*>(qt_s + 128 * 128);  // [8 warps][16][4]
-  uint32_t* col_final = col_part + kWarps * 64;             // [64]
-  uint32_t* blk_part = col_final + 64;                      // [8]
+  float* col_scale = reinterpret_cast<float*>(col_part + kWarps * 64);  // [128] 2^-e per column
+  uint32_t* blk_part = reinterpret_cast<uint32_t*>(col_scale + 128);    // [8]
   uint64_t* full = reinterpret_cast<uint64_t*>(blk_part + kWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kQStages);
 
@@ -238,18 +243,36 @@ __global__ void __launch_bounds__(kQThreads, 2)
       if (tid == 0) p.sw[tr * p.tiles_c + tc] = static_cast<uint8_t>(e_blk + 127);
     }
 
-    // ---- in-place codes (ROW, BLOCK) and the row scale bytes
+    // ---- in-place codes (ROW, BLOCK) and the row scale bytes.  Rows
+    // 8i..8i+7 share one 32-row group, so their scale bytes sit 16 apart.
     if (ROW || BLOCK) {
       uint8_t* qrow = p.q + (int64_t)(r0 + 8 * i) * p.ld_q + c0 + 8 * j;
-      // rows 8i..8i+7 share one 32-row group, so their scale bytes sit 16 apart
-      uint8_t* srow = BLOCK ? nullptr : p.s + blocked_offset(r0 + 8 * i, tc, p.s_g4);
+      if (RSHFL && !BLOCK) {
+        // thread j (< 8) of the 16 sharing rows 8i..8i+7 derives row 8i+j's
+        // exponent; the others read 2^-e from it with a shuffle
+        const int kk = j & 7;
+        const uint32_t w = rowmax[kk >> 1];
+        const int e = scale_exponent_from_bits((kk & 1) ? (w >> 16) : (w & 0xFFFFu));
+        const float s_mine = pow2_neg_x2(e).x;
+        if (j < 8) p.s[blocked_offset(r0 + 8 * i, tc, p.s_g4) + 16 * j] = static_cast<uint8_t>(e + 127);
+        const int lane16 = tid & 16;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t m = (k & 1) ? (rowmax[k >> 1] >> 16) : (rowmax[k >> 1] & 0xFFFFu);
-        const int e = BLOCK ? e_blk : scale_exponent_from_bits(m);
-        const uint2 o = encode_row8(v[k], pow2_neg_x2(e));
-        if (r0 + 8 * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
-        if (!BLOCK && j == 0) srow[16 * k] = static_cast<uint8_t>(e + 127);
+        for (int k = 0; k < 8; ++k) {
+          const float sk = __shfl_sync(0xFFFFFFFFu, s_mine, lane16 + k);
+          const uint2 o = encode_row8(v[k], make_float2(sk, sk));
+          if (r0 + 8 * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
+        }
+      } else {
+        // every thread derives the exponents of its 8 rows itself
+        uint8_t* srow = BLOCK ? nullptr : p.s + blocked_offset(r0 + 8 * i, tc, p.s_g4);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t m = (k & 1) ? (rowmax[k >> 1] >> 16) : (rowmax[k >> 1] & 0xFFFFu);
+          const int e = BLOCK ? e_blk : scale_exponent_from_bits(m);
+          const uint2 o = encode_row8(v[k], pow2_neg_x2(e));
+          if (r0 + 8 * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
+          if (!BLOCK && j == k) srow[16 * k] = static_cast<uint8_t>(e + 127);
+        }
       }
     }
 
@@ -263,27 +286,34 @@ __global__ void __launch_bounds__(kQThreads, 2)
           *reinterpret_cast<uint4*>(&col_part[(warp * 16 + j) * 4]) = make_uint4(cm[0], cm[1], cm[2], cm[3]);
         __syncthreads();
         if (tid < 64) {
+          // columns 2*tid and 2*tid+1: amax over the 8 warps, then the exponent,
+          // its scale byte (columns 8j..8j+7 sit 16 bytes apart in the blocked
+          // array) and 2^-e for every thread's encode
           uint32_t m = 0;
 #pragma unroll
           for (int w = 0; w < kWarps; ++w) m = __vmaxu2(m, col_part[(w * 16 + (tid >> 2)) * 4 + (tid & 3)]);
-          col_final[tid] = m;
+          const int e0 = scale_exponent_from_bits(m & 0xFFFFu);
+          const int e1 = scale_exponent_from_bits(m >> 16);
+          const int c = 2 * tid;
+          uint8_t* scol = p.st + blocked_offset(c0 + (c & ~7), tr, p.st_g4) + 16 * (c & 7);
+          scol[0] = static_cast<uint8_t>(e0 + 127);
+          scol[16] = static_cast<uint8_t>(e1 + 127);
+          col_scale[c] = pow2_neg_x2(e0).x;
+          col_scale[c + 1] = pow2_neg_x2(e1).x;
         }
         __syncthreads();
       }
-      const uint4 cf = *reinterpret_cast<const uint4*>(&col_final[j * 4]);
-      // columns 8j..8j+7 share one 32-row group of the blocked array: 16 bytes apart
-      uint8_t* scol = (!BLOCK && i == 0) ? p.st + blocked_offset(c0 + 8 * j, tr, p.st_g4) : nullptr;
+      float cs[8];
+      if (!BLOCK) {
+        const float4 a = *reinterpret_cast<const float4*>(&col_scale[8 * j]);
+        const float4 b = *reinterpret_cast<const float4*>(&col_scale[8 * j + 4]);
+        cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
+        cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
+      }
 #pragma unroll
       for (int l = 0; l < 8; ++l) {
-        int e;
-        if (BLOCK) {
-          e = e_blk;
-        } else {
-          const uint32_t m = word(cf, l >> 1);
-          e = scale_exponent_from_bits((l & 1) ? (m >> 16) : (m & 0xFFFFu));
-          if (i == 0) scol[16 * l] = static_cast<uint8_t>(e + 127);
-        }
-        const uint2 o = encode_col8(v, l, pow2_neg_x2(e));
+        const float2 s2 = BLOCK ? pow2_neg_x2(e_blk) : make_float2(cs[l], cs[l]);
+        const uint2 o = encode_col8(v, l, s2);
         // row (8j+l) of the transposed tile, 8-byte chunk i, XOR-swizzled by j
         *reinterpret_cast<uint2*>(qt_s + (8 * j + l) * 128 + ((i ^ j) << 3)) = o;
       }
@@ -324,7 +354,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
 // Shared memory the quantizer needs (plus alignment slack).
 constexpr uint32_t quant_smem_bytes() {
-  return kQStages * kQTileBytes + 128 * 128 + (kQThreads / 32) * 64 * 4 + 64 * 4 +
+  return kQStages * kQTileBytes + 128 * 128 + (kQThreads / 32) * 64 * 4 + 128 * 4 +
          (kQThreads / 32) * 4 + kQStages * 8 + 16 + 1024;
 }
 

@@ -35,7 +35,17 @@
 
 namespace puro {
 
-constexpr int kQThreads = 256;
+#ifndef PURO_QUANT_RPT
+#define PURO_QUANT_RPT 8
+#endif
+// rows of the 128x128 tile per thread (each thread holds RPT rows x 8 columns;
+// 16 threads cover a row, 128/RPT row groups cover the tile).  8 (256 threads,
+// two CTAs per SM) was measured faster than 4 (512 threads, 64 registers) for
+// the BOTH layout at every size tried (8192x3072: 20.9 vs 22.8 us; 16384x12288:
+// 147 vs 162 us) and equal within a few % for the single layouts.
+constexpr int kQRpt = PURO_QUANT_RPT;
+static_assert(kQRpt == 4 || kQRpt == 8, "4 or 8 rows per thread");
+constexpr int kQThreads = 16 * 128 / kQRpt;
 constexpr int kQStages = 2;
 constexpr uint32_t kQTileBytes = 128 * 128 * 2;
 
@@ -116,6 +126,12 @@ __device__ __forceinline__ uint2 encode_row8(const uint4& v, float2 s2) {
   return o;
 }
 
+// Four codes of column l of rows 0..3 of the thread's block, scaled by s2.
+__device__ __forceinline__ uint32_t encode_col4(const uint4 (&v)[4], int l, float2 s2) {
+  return encode4(make_float2(elem_f32(v[0], l), elem_f32(v[1], l)),
+                 make_float2(elem_f32(v[2], l), elem_f32(v[3], l)), s2);
+}
+
 // Eight codes of column l of the thread's 8x8 block (rows 0..7), scaled by s2.
 __device__ __forceinline__ uint2 encode_col8(const uint4 (&v)[8], int l, float2 s2) {
   uint2 o;
@@ -124,6 +140,18 @@ __device__ __forceinline__ uint2 encode_col8(const uint4 (&v)[8], int l, float2 
   o.y = encode4(make_float2(elem_f32(v[4], l), elem_f32(v[5], l)),
                 make_float2(elem_f32(v[6], l), elem_f32(v[7], l)), s2);
   return o;
+}
+
+// Column l of the thread's block as codes into its transposed-tile row `row`:
+// RPT codes at chunk i ^ (j * 8 / RPT) of RPT bytes.
+__device__ __forceinline__ void put_col_codes(uint8_t* row, const uint4 (&v)[8], int l, float2 s2,
+                                              int i, int j) {
+  *reinterpret_cast<uint2*>(row + ((i ^ j) << 3)) = encode_col8(v, l, s2);
+}
+
+__device__ __forceinline__ void put_col_codes(uint8_t* row, const uint4 (&v)[4], int l, float2 s2,
+                                              int i, int j) {
+  *reinterpret_cast<uint32_t*>(row + ((i ^ (2 * j)) << 2)) = encode_col4(v, l, s2);
 }
 
 // Larger of the two 16-bit halves.
@@ -154,6 +182,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
   uint64_t* full = reinterpret_cast<uint64_t*>(blk_part + kWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kQStages);
 
+  constexpr int RPT = kQRpt;
   const int tid = threadIdx.x;
   const int i = tid >> 4, j = tid & 15, warp = tid >> 5;
   // tiles t = blockIdx.x + it * gridDim.x, walked as (row tile, col tile)
@@ -191,11 +220,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
     const int32_t r0 = tr * 128, c0 = tc * 128;
     const int s = it % kQStages;
     const bool ok = mbar_wait(&full[s], (uint32_t)((it / kQStages) & 1), abort_flag);
-    // this thread's 8 rows x 8 columns; rows past the end were filled with 0
-    uint4 v[8];
-    const uint8_t* tile = tiles + s * kQTileBytes + (8 * i) * 256 + 16 * j;
+    // this thread's RPT rows x 8 columns; rows past the end were filled with 0
+    uint4 v[RPT];
+    const uint8_t* tile = tiles + s * kQTileBytes + (RPT * i) * 256 + 16 * j;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = ok ? lds_v4(tile + k * 256) : make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < RPT; ++k) v[k] = ok ? lds_v4(tile + k * 256) : make_uint4(0, 0, 0, 0);
     // every thread holds its part: stage s is free again (and if any wait gave
     // up, the whole block stops here together)
     if (__syncthreads_or(!ok)) break;
@@ -203,10 +232,12 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
     // ---- magnitudes: per-row amax of this thread's 8 columns (two rows per
     // word) and per-column-pair amax of its 8 rows, from the same masked words
-    uint32_t rowmax[4] = {0u, 0u, 0u, 0u};
+    uint32_t rowmax[RPT / 2];
+#pragma unroll
+    for (int q = 0; q < RPT / 2; ++q) rowmax[q] = 0u;
     uint32_t cm[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < RPT; ++k) {
       const uint32_t a0 = v[k].x & kMag, a1 = v[k].y & kMag, a2 = v[k].z & kMag,
                      a3 = v[k].w & kMag;
       if (ROW || BLOCK) {
@@ -222,7 +253,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
     }
     if (ROW || BLOCK) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < RPT / 2; ++q) {
 #pragma unroll
         for (int off = 8; off >= 1; off >>= 1)
           rowmax[q] = __vmaxu2(rowmax[q], __shfl_xor_sync(0xFFFFFFFFu, rowmax[q], off));
@@ -232,7 +263,9 @@ __global__ void __launch_bounds__(kQThreads, 2)
     int e_blk = 0;
     if (BLOCK) {
       // one exponent for the whole 128x128 block
-      uint32_t m = __vmaxu2(__vmaxu2(rowmax[0], rowmax[1]), __vmaxu2(rowmax[2], rowmax[3]));
+      uint32_t m = rowmax[0];
+#pragma unroll
+      for (int q = 1; q < RPT / 2; ++q) m = __vmaxu2(m, rowmax[q]);
       m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
       if ((tid & 31) == 0) blk_part[warp] = hmax(m);
       __syncthreads();
@@ -246,31 +279,31 @@ __global__ void __launch_bounds__(kQThreads, 2)
     // ---- in-place codes (ROW, BLOCK) and the row scale bytes.  Rows
     // 8i..8i+7 share one 32-row group, so their scale bytes sit 16 apart.
     if (ROW || BLOCK) {
-      uint8_t* qrow = p.q + (int64_t)(r0 + 8 * i) * p.ld_q + c0 + 8 * j;
+      uint8_t* qrow = p.q + (int64_t)(r0 + RPT * i) * p.ld_q + c0 + 8 * j;
       if (RSHFL && !BLOCK) {
         // thread j (< 8) of the 16 sharing rows 8i..8i+7 derives row 8i+j's
         // exponent; the others read 2^-e from it with a shuffle
-        const int kk = j & 7;
+        const int kk = j & (RPT - 1);
         const uint32_t w = rowmax[kk >> 1];
         const int e = scale_exponent_from_bits((kk & 1) ? (w >> 16) : (w & 0xFFFFu));
         const float s_mine = pow2_neg_x2(e).x;
-        if (j < 8) p.s[blocked_offset(r0 + 8 * i, tc, p.s_g4) + 16 * j] = static_cast<uint8_t>(e + 127);
+        if (j < RPT) p.s[blocked_offset(r0 + RPT * i, tc, p.s_g4) + 16 * j] = static_cast<uint8_t>(e + 127);
         const int lane16 = tid & 16;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < RPT; ++k) {
           const float sk = __shfl_sync(0xFFFFFFFFu, s_mine, lane16 + k);
           const uint2 o = encode_row8(v[k], make_float2(sk, sk));
-          if (r0 + 8 * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
+          if (r0 + RPT * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
         }
       } else {
         // every thread derives the exponents of its 8 rows itself
-        uint8_t* srow = BLOCK ? nullptr : p.s + blocked_offset(r0 + 8 * i, tc, p.s_g4);
+        uint8_t* srow = BLOCK ? nullptr : p.s + blocked_offset(r0 + RPT * i, tc, p.s_g4);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < RPT; ++k) {
           const uint32_t m = (k & 1) ? (rowmax[k >> 1] >> 16) : (rowmax[k >> 1] & 0xFFFFu);
           const int e = BLOCK ? e_blk : scale_exponent_from_bits(m);
           const uint2 o = encode_row8(v[k], pow2_neg_x2(e));
-          if (r0 + 8 * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
+          if (r0 + RPT * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
           if (!BLOCK && j == k) srow[16 * k] = static_cast<uint8_t>(e + 127);
         }
       }
@@ -313,13 +346,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
 #pragma unroll
       for (int l = 0; l < 8; ++l) {
         const float2 s2 = BLOCK ? pow2_neg_x2(e_blk) : make_float2(cs[l], cs[l]);
-        const uint2 o = encode_col8(v, l, s2);
-        // row (8j+l) of the transposed tile, 8-byte chunk i, XOR-swizzled by j
-        *reinterpret_cast<uint2*>(qt_s + (8 * j + l) * 128 + ((i ^ j) << 3)) = o;
+        // row (8j+l) of the transposed tile: this thread's RPT codes form chunk
+        // i ^ (j * 8 / RPT) of RPT bytes (the XOR spreads a warp's 16 j over
+        // distinct banks; the 16-byte readout below undoes it)
+        put_col_codes(qt_s + (8 * j + l) * 128, v, l, s2, i, j);
       }
       __syncthreads();
 #pragma unroll
-      for (int pass = 0; pass < 4; ++pass) {
+      for (int pass = 0; pass < 1024 / kQThreads; ++pass) {
         const int idx = pass * kQThreads + tid;
         const int c = idx >> 3, part = idx & 7;
         const int jj = (c >> 3) & 15;

@@ -66,19 +66,36 @@
 namespace puro {
 
 // One GEMM of a launch: D [rows_a, rows_b] (through its tm_d tensor map).
+// Its work units are its output tiles, except that tiles from split_from on
+// are each split into two half-width tiles (two units: left and right 128
+// columns), so that a last, partly-filled wave of tiles takes half as long.
 struct GemmProblem {
-  int32_t rows_a;   // output rows
-  int32_t rows_b;   // output cols
-  int32_t kblocks;  // ceil(K / BK)
+  int32_t rows_a;      // output rows
+  int32_t rows_b;      // output cols
+  int32_t kblocks;     // ceil(K / BK)
   int32_t tiles_m, tiles_n;
+  int32_t split_from;  // first split tile (== tiles_m * tiles_n: none)
+  int32_t units;       // split_from + 2 * (tiles - split_from)
 };
+
+// Tile and half (-1: whole tile, 0/1: left/right half) of a problem's unit.
+__device__ __forceinline__ void decode_unit(const GemmProblem& P, int lu, int& tile, int& h) {
+  if (lu < P.split_from) {
+    tile = lu;
+    h = -1;
+  } else {
+    const int d = lu - P.split_from;
+    tile = P.split_from + (d >> 1);
+    h = d & 1;
+  }
+}
 
 constexpr int kMaxSchedClusters = 128;
 constexpr int kMaxSchedUnits = 2048;
 
 // A launch computes one or two independent GEMMs (the data and weight
-// gradients of one layer share a launch).  Its work units are the output tiles:
-// units [0, tiles0) are problem 0's tiles, the rest problem 1's.  Clusters take
+// gradients of one layer share a launch).  Units [0, tiles0) are problem 0's,
+// the rest problem 1's.  Clusters take
 // units either round robin (unit u -> cluster u % clusters) or from a host-made
 // schedule: cluster c runs sched_unit[sched_off[c] .. sched_off[c+1]) in order.
 struct GemmParams {
@@ -158,6 +175,10 @@ struct GemmCfg {
   static constexpr uint32_t kIdesc =
       ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(kBM >> 4) << 24);
   static constexpr uint32_t kTxPerStage = CG * (kABytes + kBBytes);
+  // half-width tiles (BN/2 output columns: N = BN/2 MMAs, half the B rows)
+  static constexpr uint32_t kIdescHalf =
+      ((uint32_t)((BN / 2) >> 3) << 17) | (1u << 23) | ((uint32_t)(kBM >> 4) << 24);
+  static constexpr uint32_t kTxPerStageHalf = CG * (kABytes + kBBytes / 2);
   static constexpr uint32_t kTxPerSf = CG * kSfSlotBytes;
 };
 
@@ -228,6 +249,8 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
                              const __grid_constant__ CUtensorMap tm_sfa1,
                              const __grid_constant__ CUtensorMap tm_sfb1,
                              const __grid_constant__ CUtensorMap tm_d1,
+                             const __grid_constant__ CUtensorMap tm_bh0,
+                             const __grid_constant__ CUtensorMap tm_bh1,
                              const __grid_constant__ GemmParams p) {
   using C = GemmCfg<CG, BN, BK>;
   constexpr int S = C::kStages;
@@ -274,6 +297,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     prefetch_tmap(&tm_sfa0);
     prefetch_tmap(&tm_sfb0);
     prefetch_tmap(&tm_d0);
+    prefetch_tmap(&tm_bh0);
     if (p.nprob > 1) {
       prefetch_tmap(&tm_a1);
       prefetch_tmap(&tm_b1);
@@ -304,15 +328,19 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     for (int ui = 0; ui < nunits && ok; ++ui) {
       const int u = unit_at(p, cluster_id, num_clusters, ui);
       const int pr = u >= p.tiles0 ? 1 : 0;
-      const int tile = u - (pr ? p.tiles0 : 0);
       const GemmProblem& P = p.prob[pr];
+      int tile, h;
+      decode_unit(P, u - (pr ? p.tiles0 : 0), tile, h);
+      const bool halft = h >= 0;
       const CUtensorMap* tm_a = pr ? &tm_a1 : &tm_a0;
-      const CUtensorMap* tm_b = pr ? &tm_b1 : &tm_b0;
+      const CUtensorMap* tm_b = halft ? (pr ? &tm_bh1 : &tm_bh0) : (pr ? &tm_b1 : &tm_b0);
       const CUtensorMap* tm_sfa = pr ? &tm_sfa1 : &tm_sfa0;
       const CUtensorMap* tm_sfb = pr ? &tm_sfb1 : &tm_sfb0;
       const int tm = tile % P.tiles_m, tn = tile / P.tiles_m;
       const int a_row = tm * C::kBM + 128 * (int)rank;
-      const int b_row = tn * BN + C::kBNC * (int)rank;
+      const int b_col0 = tn * BN + (halft ? (BN / 2) * h : 0);   // first output column
+      const int b_row = b_col0 + (halft ? C::kBNC / 2 : C::kBNC) * (int)rank;
+      const uint32_t tx = halft ? C::kTxPerStageHalf : C::kTxPerStage;
       for (int kb = 0; kb < P.kblocks; ++kb) {
         if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
         const bool sf = (kb % C::kStagesPerSf) == 0;
@@ -320,7 +348,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
         if (sf && !mbar_wait_warp(&sfe[slot], ((sfc / R) & 1) ^ 1, abort_flag)) { ok = false; break; }
         if (elect_one()) {
           if (leader)
-            mbar_arrive_expect_tx(&full[stage], C::kTxPerStage + (sf ? C::kTxPerSf : 0u));
+            mbar_arrive_expect_tx(&full[stage], tx + (sf ? C::kTxPerSf : 0u));
           const uint32_t bar = leader_addr<CG>(&full[stage]);
           tma_load_2d<CG>(smem + C::kOffA + stage * C::kABytes, tm_a, kb * BK, a_row, bar);
           tma_load_2d<CG>(smem + C::kOffB + stage * C::kBBytes, tm_b, kb * BK, b_row, bar);
@@ -328,7 +356,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
             uint8_t* sfbuf = smem + C::kOffSf + slot * C::kSfSlotBytes;
             const int chunk = kb / C::kStagesPerSf;
             tma_load_3d<CG>(sfbuf, tm_sfa, 0, chunk, a_row >> 7, bar);
-            tma_load_3d<CG>(sfbuf + C::kSfaBytes, tm_sfb, 0, chunk, (tn * BN) >> 7, bar);
+            tma_load_3d<CG>(sfbuf + C::kSfaBytes, tm_sfb, 0, chunk, b_col0 >> 7, bar);
           }
         }
         if (sf) ++sfc;
@@ -357,7 +385,11 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       const uint64_t bdesc0 = desc_kmajor<BK>(smem_u32(smem + C::kOffB));
       for (int ui = 0; ui < nunits && ok; ++ui, ++it) {
         const int u = unit_at(p, cluster_id, num_clusters, ui);
-        const int kblocks = p.prob[u >= p.tiles0 ? 1 : 0].kblocks;
+        const int pr = u >= p.tiles0 ? 1 : 0;
+        const int kblocks = p.prob[pr].kblocks;
+        int tile_unused, h;
+        decode_unit(p.prob[pr], u - (pr ? p.tiles0 : 0), tile_unused, h);
+        const uint32_t idesc_base = h >= 0 ? C::kIdescHalf : C::kIdesc;
         const int acc = it % NA;
         const uint32_t acc_phase = (it / NA) & 1;
         if (!mbar_wait_warp(&acce[acc], acc_phase ^ 1, abort_flag)) break;
@@ -390,7 +422,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
           if (elect_one()) {
             const uint32_t t_sf = t_sfreg + 16 * ((sfc - 1) & 1);
             const uint32_t j = (uint32_t)((kb / C::kSub) & 3);  // 128-group within the chunk
-            const uint32_t idesc = C::kIdesc | (j << 29) | (j << 4);
+            const uint32_t idesc = idesc_base | (j << 29) | (j << 4);
             // start-address field (16-byte units) of the stage's descriptors
             const uint64_t adesc = adesc0 + (uint64_t)(stage * (C::kABytes >> 4));
             const uint64_t bdesc = bdesc0 + (uint64_t)(stage * (C::kBBytes >> 4));
@@ -421,8 +453,9 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
     for (int ui = 0; ui < nunits; ++ui, ++it) {
       const int u = unit_at(p, cluster_id, num_clusters, ui);
       const int pr = u >= p.tiles0 ? 1 : 0;
-      const int tile = u - (pr ? p.tiles0 : 0);
       const GemmProblem& P = p.prob[pr];
+      int tile, h;
+      decode_unit(P, u - (pr ? p.tiles0 : 0), tile, h);
       const int tm = tile % P.tiles_m, tn = tile / P.tiles_m;
       const int acc = it % NA;
       const uint32_t acc_phase = (it / NA) & 1;
@@ -458,11 +491,15 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_leader<CG>(&acce[acc]);
       const int row0 = tm * C::kBM + 128 * (int)rank + sp * 32;
-      const int gcol = tn * BN + half * C::kEpiCols;
-      if (pr == 0)
-        epilogue_store<C, OUT0>(r, &tm_d0, ebuf, ebufc, lane, row0, gcol, P.rows_a, P.rows_b);
-      else
-        epilogue_store<C, OUT1>(r, &tm_d1, ebuf, ebufc, lane, row0, gcol, P.rows_a, P.rows_b);
+      // a half-width unit has BN/2 valid accumulator columns (the MMA wrote only
+      // those; the rest were loaded above for the tail hand-over and are dropped)
+      const int gcol = tn * BN + (h >= 0 ? (BN / 2) * h : 0) + half * C::kEpiCols;
+      if (h < 0 || half * C::kEpiCols < BN / 2) {
+        if (pr == 0)
+          epilogue_store<C, OUT0>(r, &tm_d0, ebuf, ebufc, lane, row0, gcol, P.rows_a, P.rows_b);
+        else
+          epilogue_store<C, OUT1>(r, &tm_d1, ebuf, ebufc, lane, row0, gcol, P.rows_a, P.rows_b);
+      }
     }
     // the staging buffers must stay valid until the stores have read them
     if (lane == 0) bulk_wait_group<0>();

@@ -185,7 +185,8 @@ struct GemmArgs {
   int out;                          // puro::GemmOut
 };
 
-// Tensor maps of one GEMM: operands, their scales and the output.
+// Tensor maps of one GEMM: A, B, the scales of A and B, the output, and B
+// again with half-height boxes (m[0..5]).
 template <int CG, int BN, int BK, int OUT>
 int make_gemm_maps(const GemmArgs& g, CUtensorMap* m) {
   using C = puro::GemmCfg<CG, BN, BK>;
@@ -194,6 +195,8 @@ int make_gemm_maps(const GemmArgs& g, CUtensorMap* m) {
   const CUtensorMapSwizzle sw = BK == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if ((st = make_map_u8(&m[0], g.a, g.k, g.rows_a, g.lda, BK, 128, sw)) != PURO_OK) return st;
   if ((st = make_map_u8(&m[1], g.b, g.k, g.rows_b, g.ldb, BK, C::kBNC, sw)) != PURO_OK) return st;
+  // B in half-height boxes, for half-width tiles
+  if ((st = make_map_u8(&m[5], g.b, g.k, g.rows_b, g.ldb, BK, C::kBNC / 2, sw)) != PURO_OK) return st;
   if ((st = make_map_scales(&m[2], g.sfa, g.rows_a, kb, 1)) != PURO_OK) return st;
   if ((st = make_map_scales(&m[3], g.sfb, g.rows_b, kb, C::kNB)) != PURO_OK) return st;
   // output [rows_a, rows_b], row stride ldd elements; store boxes of 32 rows
@@ -218,7 +221,7 @@ void make_schedule(puro::GemmParams& p, int clusters) {
   const int units = p.units;
   std::vector<int> order(units);
   for (int u = 0; u < units; ++u) order[u] = u;
-  auto cost = [&](int u) { return p.prob[u >= p.tiles0 ? 1 : 0].kblocks + 2; };
+  auto cost = [&](int u) { return p.prob[u >= p.tiles0 ? 1 : 0].kblocks + 2; };  // no split units here
   std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return cost(x) > cost(y); });
   using Slot = std::pair<int64_t, int>;  // (load, cluster), least load first, then lowest index
   std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
@@ -244,7 +247,7 @@ void make_schedule(puro::GemmParams& p, int clusters) {
 template <int CG, int BN, int BK, int OUT0, int OUT1>
 int launch_gemm_cfg(const GemmArgs& g0, const GemmArgs* g1, DeviceInfo* dev, cudaStream_t stream) {
   using C = puro::GemmCfg<CG, BN, BK>;
-  CUtensorMap m0[5], m1[5];
+  CUtensorMap m0[6], m1[6];
   int st;
   if ((st = make_gemm_maps<CG, BN, BK, OUT0>(g0, m0)) != PURO_OK) return st;
   if (g1) {
@@ -290,16 +293,30 @@ int launch_gemm_cfg(const GemmArgs& g0, const GemmArgs* g1, DeviceInfo* dev, cud
     p.prob[i].tiles_m = (int32_t)((g.rows_a + C::kBM - 1) / C::kBM);
     p.prob[i].tiles_n = (int32_t)((g.rows_b + BN - 1) / BN);
   }
-  const int64_t t0 = (int64_t)p.prob[0].tiles_m * p.prob[0].tiles_n;
-  const int64_t t1 = g1 ? (int64_t)p.prob[1].tiles_m * p.prob[1].tiles_n : 0;
-  p.tiles0 = (int32_t)t0;
-  p.units = (int32_t)(t0 + t1);
-  const int clusters = p.units < max_clusters[dev_id] ? p.units : max_clusters[dev_id];
+  const int C_max = max_clusters[dev_id];
+  for (int i = 0; i < p.nprob; ++i) {
+    const int64_t t = (int64_t)p.prob[i].tiles_m * p.prob[i].tiles_n;
+    p.prob[i].split_from = (int32_t)t;
+    p.prob[i].units = (int32_t)t;
+  }
+  if (!g1 && BN == 256) {
+    // one GEMM: if the last wave of tiles would fill at most half the clusters,
+    // split its tiles into half-width tiles, which then all run at once
+    const int64_t t = p.prob[0].split_from;
+    const int64_t full = (t / C_max) * C_max, rest = t - full;
+    if (rest > 0 && 2 * rest <= C_max) {
+      p.prob[0].split_from = (int32_t)full;
+      p.prob[0].units = (int32_t)(full + 2 * rest);
+    }
+  }
+  p.tiles0 = p.prob[0].units;
+  p.units = p.prob[0].units + (g1 ? p.prob[1].units : 0);
+  const int clusters = p.units < C_max ? p.units : C_max;
   if (g1 && p.units <= puro::kMaxSchedUnits) make_schedule(p, clusters);
   cfg.gridDim = dim3(CG * clusters);
   cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, kern, m0[0], m0[1], m0[2], m0[3], m0[4], m1[0], m1[1], m1[2], m1[3],
-                         m1[4], p) != cudaSuccess)
+                         m1[4], m0[5], m1[5], p) != cudaSuccess)
     return PURO_ERR_CUDA;
   return launch_status();
 }

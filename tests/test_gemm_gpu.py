@@ -145,3 +145,27 @@ def test_dgrad_wgrad_launch_matches_separate_calls(fp8, m, n, k, kind):
     assert torch.equal(dx.view(torch.int16), dx_ref.view(torch.int16))
     assert torch.equal(dw.view(torch.int16 if kind == "bf16" else torch.int32),
                        dw_ref.view(torch.int16 if kind == "bf16" else torch.int32))
+
+
+def test_half_width_tail_tiles_match_whole_tiles(fp8, oracle_mod):
+    """A launch whose last wave would fill at most half the clusters splits
+    those tiles into two half-width tiles.  Every output element is still one
+    K loop in the same order: the split result equals, bit for bit, the same
+    rows computed in a launch that does not split (more rows, full waves)."""
+    clusters = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    n, k = 512, 384
+    m_split = 256 * ((clusters + 1) // 2 + 1)     # 2 * tiles_m tiles -> one full wave + a few
+    m_full = 256 * clusters                         # 2 * clusters tiles: whole waves, no split
+    g = torch.Generator().manual_seed(77)
+    x = torch.randn(m_full, k, generator=g).to(torch.bfloat16)
+    w = (torch.randn(n, k, generator=g) * 0.02).to(torch.bfloat16)
+    dev = torch.device("cuda")
+    wq = fp8.quant_weight(w.to(dev))
+    y_full = fp8.gemm_fprop(fp8.quant_act(x.to(dev), "rowwise"), wq)
+    y_split = fp8.gemm_fprop(fp8.quant_act(x[:m_split].to(dev), "rowwise"), wq)
+    torch.cuda.synchronize()
+    assert fp8.device_status() == 0
+    assert torch.equal(y_split.view(torch.int16), y_full[:m_split].view(torch.int16))
+    rows = np.unique(np.linspace(0, m_split - 1, 24).astype(np.int64))
+    assert_gemm_close(y_split[rows.tolist()], oracle_mod.linear_fprop(x[rows], w), oracle_mod,
+                      "split-tail fprop")

@@ -3,9 +3,10 @@
 One step = one micro-batch of the attention-projection workload (M = 8192
 tokens, hidden 2048; the fused QKV projection 2048->3072 and the output
 projection 2048->2048), for each of the two layers:
-  quant_weight(W) (+ transposed codes), quant_act(X, both), fprop,
-  quant_act(dY, both), and one launch computing dgrad and wgrad (dW added
-  into FP32 main grads).
+  quant_act(X, both), fprop, quant_act(dY, both), and one launch computing
+  dgrad and wgrad (dW added into FP32 main grads); quant_weight(W) (+
+  transposed codes) runs once per gradient-accumulation window of --accum
+  steps, since the weights only change at the optimizer step.
 value = GEMM FLOPs of the step (2*M*N*K per GEMM, three GEMMs per layer)
 divided by the device time of the whole step (quantizers included).
 
@@ -150,13 +151,21 @@ class Step:
         # its dW into it (one micro-batch of gradient accumulation)
         self.grads = MainGrads([(w.shape[0], w.shape[1]) for (_, w, _) in self.sets[0]], device=dev)
         torch.cuda.synchronize()
-        self.names = []
-        for L in wl.layers:
-            self.names += ["%s.quant_weight" % L.name, "%s.quant_x" % L.name, "%s.fprop" % L.name,
-                           "%s.quant_dy" % L.name, "%s.dgrad_wgrad" % L.name]
-        self.launches_per_step = len(self.names)
+        self.all_names = self.launch_names(True)
 
-    def run(self, set_idx, events=None):
+    def launch_names(self, weights):
+        names = []
+        for L in self.layers:
+            if weights:
+                names.append("%s.quant_weight" % L.name)
+            names += ["%s.quant_x" % L.name, "%s.fprop" % L.name, "%s.quant_dy" % L.name,
+                      "%s.dgrad_wgrad" % L.name]
+        return names
+
+    def run(self, set_idx, events=None, weights=True):
+        """One micro-batch step.  The weights are quantized only when `weights`:
+        within a gradient-accumulation window they do not change, so the first
+        step's codes serve the whole window."""
         fp8 = self.fp8
         ev = iter(events) if events is not None else None
 
@@ -165,7 +174,8 @@ class Step:
                 next(ev).record()
 
         for li, ((x, w, dy), (xq, wq, dyq, y, dx)) in enumerate(zip(self.sets[set_idx], self.out)):
-            mark(); fp8.quant_weight(w, transpose=True, out=wq); mark()
+            if weights:
+                mark(); fp8.quant_weight(w, transpose=True, out=wq); mark()
             mark(); fp8.quant_act(x, "both", out=xq); mark()
             mark(); fp8.gemm_fprop(xq, wq, out=y); mark()
             mark(); fp8.quant_act(dy, "both", out=dyq); mark()
@@ -210,8 +220,9 @@ def run_ours(args):
     step = Step(wl, dev)
     costs = _unit_costs(wl)
     gemm_flops = wl.gemm_flops()
+    A = max(1, min(args.accum, args.steps))
     for i in range(args.warmup):
-        step.run(i % len(step.sets))
+        step.run(i % len(step.sets), weights=(i % A == 0))
     torch.cuda.synchronize()
     status = step.fp8.device_status()
     if status != 0:
@@ -228,12 +239,11 @@ def run_ours(args):
     # programmatic (PDL) edges that let a kernel's prologue overlap its
     # predecessor's tail.
     K = args.steps
-    A = max(1, min(args.accum, K))
     windows = [A] * (K // A) + ([K % A] if K % A else [])
-    nl = step.launches_per_step
     K_inst = min(K, 100)
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * nl)]
-          for _ in range(K_inst)]
+    inst_names = [step.launch_names(i % A == 0) for i in range(K_inst)]
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * len(nm))]
+          for nm in inst_names]
     graphs = {}
     graph_inst = torch.cuda.CUDAGraph()
     cap_stream = torch.cuda.Stream()
@@ -243,10 +253,10 @@ def run_ours(args):
             graphs[n] = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graphs[n], stream=cap_stream):
                 for i in range(n):
-                    step.run(i % len(step.sets))
+                    step.run(i % len(step.sets), weights=(i == 0))
         with torch.cuda.graph(graph_inst, stream=cap_stream):
             for i in range(K_inst):
-                step.run(i % len(step.sets), ev[i])
+                step.run(i % len(step.sets), ev[i], weights=(i % A == 0))
     torch.cuda.synchronize()
     for g in graphs.values():  # untimed first replays of the instantiated graphs
         g.replay()
@@ -276,10 +286,11 @@ def run_ours(args):
     clocks = clk.summary()
 
     total_ms = t_start.elapsed_time(t_end)
-    per_launch = {name: [] for name in step.names}
+    per_launch = {name: [] for name in step.all_names}
     for i in range(K_inst):
-        for j, name in enumerate(step.names):
+        for j, name in enumerate(inst_names[i]):
             per_launch[name].append(ev[i][2 * j].elapsed_time(ev[i][2 * j + 1]))
+    launches_timed = sum(n * len(step.launch_names(False)) + len(step.layers) for n in windows)
     ms_per_step = total_ms / K
     if world > 1:
         t = torch.tensor([ms_per_step], device=dev)
@@ -291,13 +302,14 @@ def run_ours(args):
     fp8_peak_tf = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     value = gemm_flops * world / (ms_per_step * 1e-3) / 1e12
 
-    gemm_ms = sum(statistics.mean(per_launch[n]) for n in step.names if costs[n][0] == "flops")
+    gemm_ms = sum(statistics.mean(per_launch[n]) for n in step.all_names if costs[n][0] == "flops")
     gemm_tf = gemm_flops / (gemm_ms * 1e-3) / 1e12
-    quant_ms = sum(statistics.mean(per_launch[n]) for n in step.names if costs[n][0] == "bytes")
-    quant_bytes = sum(costs[n][1] for n in step.names if costs[n][0] == "bytes")
+    # quantizer bandwidth over every quantizer launch of the instrumented replay
+    quant_ms = sum(sum(per_launch[n]) for n in step.all_names if costs[n][0] == "bytes")
+    quant_bytes = sum(costs[n][1] * len(per_launch[n]) for n in step.all_names if costs[n][0] == "bytes")
     quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
     breakdown = {}
-    for n in step.names:
+    for n in step.all_names:
         kind, amount = costs[n]
         ms = statistics.mean(per_launch[n])
         rate = amount / (ms * 1e-3) / (1e12 if kind == "flops" else 1e9)
@@ -305,7 +317,7 @@ def run_ours(args):
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(wl, dev, K=min(K, 10), warmup=2)
+        e2e = run_e2e(wl, dev, K=min(K, 10), warmup=2, accum=A)
         if world > 1:
             t = torch.tensor([e2e["ms_per_step"]], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -354,8 +366,9 @@ def run_ours(args):
                 "global_batch_tokens": M_TOKENS * world,
                 "l2": "3 rotating input sets of 132 MB each (> 126 MB L2)",
                 "parallelism": "dp%d (own batch per rank; FP32 dW all-reduce every %d steps)" % (world, A),
-                "step": "per layer: quant_weight, quant_act(X), fprop, quant_act(dY), and one "
-                        "launch for dgrad + wgrad (dW added into FP32 main grads)",
+                "step": "per layer: quant_act(X), fprop, quant_act(dY), and one launch for "
+                        "dgrad + wgrad (dW added into FP32 main grads); quant_weight once per "
+                        "%d-step accumulation window (the weights do not change within it)" % A,
                 "grad_exchange": "every %d steps: FP32 dW all-reduce across ranks (NCCL) and clear"
                                  % A,
             },
@@ -376,7 +389,7 @@ def run_ours(args):
                 "peak": peaks["hbm_gbs"], "frac": round(quant_gbs / peaks["hbm_gbs"], 4),
             },
             "kernels": breakdown,
-            "gpu_launches": step.launches_per_step * K,
+            "gpu_launches": launches_timed,
             "clocks": clocks,
             "wall_ms_timed_region": round(total_ms, 3),
             "timing": "K steps as CUDA graphs of %d steps plus the gradient exchange between them "
@@ -521,30 +534,34 @@ def fp8_ceiling(wl, dev):
         return {"unavailable": str(e).splitlines()[0][:160]}
 
 
-def run_e2e(wl, dev, K, warmup):
-    """Same step through the public API with pinned host inputs/outputs: every
-    step copies X, W, dY in, runs forward and backward (dW added into the FP32
-    main grads), and copies Y, dX and the main grads back, all inside the
-    timed region.  The copies are pipelined across steps the way a training
-    loop would: step i+1's inputs go up on a copy stream while step i
-    computes, and step i's results come down on another while step i+1
-    computes (double-buffered device and host buffers, ordered by events)."""
+def run_e2e(wl, dev, K, warmup, accum):
+    """Same step through the public API with pinned host inputs/outputs, inside
+    the timed region: every step copies X and dY in (and, at the start of each
+    `accum`-step accumulation window, W, which is then quantized once for the
+    window), runs forward and backward (dW added into the FP32 main grads),
+    and copies Y, dX and the main grads back.  The copies are pipelined across
+    steps the way a training loop would: step i+1's inputs go up on a copy
+    stream while step i computes, and step i's results come down on another
+    while step i+1 computes (double-buffered buffers, ordered by events)."""
     import torch
     import fp8_block_scaled_13_b200 as fp8
     from fp8_block_scaled_13_b200.dp import MainGrads
 
     nbuf = 2
-    host_in = [[(L.x.pin_memory(), L.w.pin_memory(), L.dy.pin_memory()) for L in wl.layers]
-               for _ in range(nbuf)]
+    host_w = [L.w.pin_memory() for L in wl.layers]
+    host_in = [[(L.x.pin_memory(), L.dy.pin_memory()) for L in wl.layers] for _ in range(nbuf)]
     host_out = [[(torch.empty((L.m, L.n), dtype=torch.bfloat16).pin_memory(),
                   torch.empty((L.m, L.k), dtype=torch.bfloat16).pin_memory(),
                   torch.empty((L.n, L.k), dtype=torch.float32).pin_memory()) for L in wl.layers]
                 for _ in range(nbuf)]
-    dev_in = [[(torch.empty_like(x, device=dev), torch.empty_like(w, device=dev),
-                torch.empty_like(dy, device=dev)) for (x, w, dy) in host_in[0]] for _ in range(nbuf)]
+    dev_w = [torch.empty_like(w, device=dev) for w in host_w]
+    dev_in = [[(torch.empty_like(x, device=dev), torch.empty_like(dy, device=dev))
+               for (x, dy) in host_in[0]] for _ in range(nbuf)]
+    wq = [None] * len(wl.layers)
     results = [None] * nbuf   # device outputs (Y, dX) of the step that used buffer b
     grads = [MainGrads([(L.n, L.k) for L in wl.layers], device=dev) for _ in range(nbuf)]
-    h2d = sum(t.numel() * t.element_size() for tup in host_in[0] for t in tup)
+    bytes_w = sum(t.numel() * t.element_size() for t in host_w)
+    bytes_in = sum(t.numel() * t.element_size() for tup in host_in[0] for t in tup)
     d2h = sum(t.numel() * t.element_size() for tup in host_out[0] for t in tup)
     comp = torch.cuda.current_stream()
     up = torch.cuda.Stream()
@@ -556,10 +573,13 @@ def run_e2e(wl, dev, K, warmup):
     def upload(i):
         b = i % nbuf
         with torch.cuda.stream(up):
-            up.wait_event(ev_done[b])   # the previous use of these device inputs is over
-            for (hx, hw, hdy), (x, w, dy) in zip(host_in[b], dev_in[b]):
+            up.wait_event(ev_done[b])   # the previous use of these device buffers is over
+            if i % accum == 0:
+                up.wait_event(ev_done[(i - 1) % nbuf])   # the last user of the old weights
+                for hw, w in zip(host_w, dev_w):
+                    w.copy_(hw, non_blocking=True)
+            for (hx, hdy), (x, dy) in zip(host_in[b], dev_in[b]):
                 x.copy_(hx, non_blocking=True)
-                w.copy_(hw, non_blocking=True)
                 dy.copy_(hdy, non_blocking=True)
             ev_up[b].record(up)
 
@@ -568,9 +588,12 @@ def run_e2e(wl, dev, K, warmup):
         comp.wait_event(ev_up[b])
         comp.wait_event(ev_down[b])   # the previous results of buffer b went down
         outs = []
-        for li, (x, w, dy) in enumerate(dev_in[b]):
-            y, xq, wq = fp8.linear_forward(x, w)
-            dx, _ = fp8.linear_backward(dy, xq, wq, main_grad=grads[b][li])
+        for li, (x, dy) in enumerate(dev_in[b]):
+            if i % accum == 0:
+                y, xq, wq[li] = fp8.linear_forward(x, dev_w[li])
+            else:
+                y, xq, _ = fp8.linear_forward(x, wq=wq[li])
+            dx, _ = fp8.linear_backward(dy, xq, wq[li], main_grad=grads[b][li])
             y.record_stream(down)
             dx.record_stream(down)
             outs.append((y, dx))
@@ -604,7 +627,9 @@ def run_e2e(wl, dev, K, warmup):
     run(K)
     e.record()
     torch.cuda.synchronize()
-    return {"ms_per_step": s.elapsed_time(e) / K, "h2d": h2d, "d2h": d2h}
+    windows = (K + accum - 1) // accum
+    return {"ms_per_step": s.elapsed_time(e) / K,
+            "h2d": int(bytes_in + bytes_w * windows / K), "d2h": d2h}
 
 
 # ---------------------------------------------------------------- CPU oracle

@@ -223,10 +223,18 @@ def device_status() -> int:
     return _lib.puro_fp8_device_status(_stream())
 
 
-def linear_forward(x: torch.Tensor, w: torch.Tensor):
-    """Quantize X and W, then Y = X W^T.  Returns (y, xq, wq)."""
+def linear_forward(x: torch.Tensor, w: torch.Tensor | None = None, wq: QuantWeight | None = None):
+    """Quantize X (and W, unless its quantization `wq` is passed in), then
+    Y = X W^T.  Returns (y, xq, wq).
+
+    Passing the previous call's `wq` skips re-quantizing a weight that has not
+    changed, e.g. across the micro-batches of one gradient-accumulation step
+    (the codes would be identical)."""
+    if wq is None:
+        if w is None:
+            raise ValueError("pass the weight or its quantization")
+        wq = quant_weight(w, transpose=True)
     xq = quant_act(x, "both")
-    wq = quant_weight(w, transpose=True)
     return gemm_fprop(xq, wq), xq, wq
 
 

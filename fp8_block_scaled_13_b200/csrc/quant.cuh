@@ -236,13 +236,19 @@ __global__ void __launch_bounds__(kQThreads, 2)
 #pragma unroll
     for (int q = 0; q < RPT / 2; ++q) rowmax[q] = 0u;
     uint32_t cm[4] = {0u, 0u, 0u, 0u};
+    uint32_t even_row = 0u;  // (even, odd)-column maxima of the last even row
 #pragma unroll
     for (int k = 0; k < RPT; ++k) {
       const uint32_t a0 = v[k].x & kMag, a1 = v[k].y & kMag, a2 = v[k].z & kMag,
                      a3 = v[k].w & kMag;
       if (ROW || BLOCK) {
-        const uint32_t m = hmax(__vmaxu2(__vmaxu2(a0, a1), __vmaxu2(a2, a3)));
-        rowmax[k >> 1] |= (k & 1) ? (m << 16) : m;
+        // two rows per word: the low halves of rows k-1, k side by side, the
+        // high halves side by side, and one packed max of the two
+        const uint32_t t = __vmaxu2(__vmaxu2(a0, a1), __vmaxu2(a2, a3));
+        if (k & 1)
+          rowmax[k >> 1] = __vmaxu2(__byte_perm(even_row, t, 0x5410), __byte_perm(even_row, t, 0x7632));
+        else
+          even_row = t;
       }
       if (COL && !BLOCK) {
         cm[0] = __vmaxu2(cm[0], a0);

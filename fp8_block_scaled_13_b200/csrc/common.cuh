@@ -159,11 +159,18 @@ __device__ __forceinline__ uint32_t leader_addr(const void* p) {
   return a;
 }
 
-// Arrive once on `bar` in the leader CTA (release at cluster scope).
+// Arrive once on `bar` in the leader CTA, for hand-overs that only order
+// tcgen05 (TMEM) accesses: the arriving warp ends its TMEM reads with
+// tcgen05.wait::ld + tcgen05.fence::before_thread_sync and the waiting warp
+// starts with tcgen05.fence::after_thread_sync, so the arrive itself carries
+// the default CTA-scope release.  (A cluster-scope release was measured at
+// 1.2-2.0 k cycles here -- it also waits for this thread's earlier memory
+// operations, including in-flight TMA stores -- and sat on the tile-to-tile
+// critical path.)
 template <int CG>
 __device__ __forceinline__ void mbar_arrive_leader(uint64_t* bar) {
   const uint32_t a = leader_addr<CG>(bar);
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(a) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(a) : "memory");
 }
 
 // ---------------------------------------------------------------- TMA

@@ -163,7 +163,7 @@ struct GemmCfg {
   static constexpr uint32_t kOffSf = kOffB + kStages * kBBytes;
   static constexpr uint32_t kOffEpi = (kOffSf + kSfSlots * kSfSlotBytes + 1023) / 1024 * 1024;
   static constexpr uint32_t kOffBar = kOffEpi + kEpiBytes;
-  static constexpr uint32_t kNumBars = 2 * kStages + kSfSlots + 3 * kNacc + 1;
+  static constexpr uint32_t kNumBars = 2 * kStages + kSfSlots + 4 * kNacc + 1;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -267,6 +267,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
   uint64_t* acce = bars + 2 * S + R + NA;
   uint64_t* drain = bars + 2 * S + R + 2 * NA;
   uint64_t* sft = bars + 2 * S + R + 2 * NA + 1;  // accumulator tail (scale area) drained
+  uint64_t* tld = sft + NA;                        // this CTA's tail loads done (local)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -288,6 +289,7 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       mbar_init(&accf[a], 1);
       mbar_init(&acce[a], C::kEpiWarps * CG);
       mbar_init(&sft[a], (C::kEpiWarps / 2) * CG);
+      mbar_init(&tld[a], C::kEpiWarps / 2);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -466,13 +468,19 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       uint32_t r[C::kEpiCols];
       constexpr int NC = C::kEpiCols / 32;
       if (C::kSfInTail && half == 1) {
-        // the last 32 columns first: the next tile's scales go there
+        // the last 32 columns first: the next tile's scales go there.  The
+        // other warp of this sub-partition holds its own loads back until
+        // these have completed (barrier tld), so the hand-over is not queued
+        // behind 128 columns of its loads.
         tmem_ld_32x32b_x32(t_base + (NC - 1) * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[(NC - 1) * 32]));
         tmem_ld_wait();
         regs_after_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[(NC - 1) * 32]));
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_leader<CG>(&sft[acc]);
+        if (lane == 0) {
+          mbar_arrive_leader<CG>(&sft[acc]);
+          mbar_arrive(&tld[acc]);
+        }
 #pragma unroll
         for (int c = 0; c < NC - 1; ++c)
           tmem_ld_32x32b_x32(t_base + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
@@ -480,6 +488,9 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < NC - 1; ++c) regs_after_wait(*reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
       } else {
+        // (per-accumulator barrier: its phase cannot run two tiles ahead of
+        // this wait, since that tile's MMAs need this warp's release below)
+        if (C::kSfInTail && !mbar_wait(&tld[acc], acc_phase, abort_flag)) break;
 #pragma unroll
         for (int c = 0; c < NC; ++c)
           tmem_ld_32x32b_x32(t_base + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));

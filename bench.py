@@ -37,7 +37,7 @@ M_TOKENS = 8192
 # dram__bytes_read.sum + dram__bytes_write.sum of one GEMM launch (fprop, QKV
 # layer) from the ncu capture summarised in profiles/; None until captured
 # for the current kernel.
-GEMM_TRAFFIC_BYTES = 23327744 + 6664960  # QKV fprop launch, profiles/gemm_block_scaled_attn_proj_qkv_fprop.md
+GEMM_TRAFFIC_BYTES = 23338496 + 6511104  # QKV fprop launch, profiles/gemm_block_scaled_attn_proj_qkv_fprop.md
 
 
 def _peaks():

@@ -7,7 +7,10 @@
 // along the reduction dimension for activations and gradients, 128x128 blocks
 // for weights -- paper.rainbus.top "方法步骤详情" step (3), ta-paperlens §3.2).
 // fprop, dgrad and wgrad are all this one contraction with different operands
-// (see the host entry points).  FP32 accumulation in TMEM, BF16 output (RNE).
+// (see the host entry points).  FP32 accumulation in TMEM; BF16 (RNE) or FP32
+// output.  A launch computes one GEMM, or two independent ones (a layer's
+// data and weight gradients), over one list of output-tile work units that
+// the clusters take round robin or from a host-made schedule (GemmParams).
 //
 // The pages' "Blackwell MXFP8 path" maps onto tcgen05.mma kind::mxf8f6f4 with
 // block scaling: the MMA multiplies each 32-element K slice by one UE8M0 scale

@@ -40,6 +40,30 @@ def _check(status: int, where: str):
         raise _lib.PuroError(status, where)
 
 
+def _need(t, what: str):
+    if t is None:
+        raise ValueError(what)
+    return t
+
+
+def _check_tensor(t: torch.Tensor, shape, dtypes, name: str, min_cols: bool = False):
+    """A caller-supplied buffer: CUDA, one of `dtypes`, row-major 2-D of
+    `shape` (with min_cols: at least shape[1] columns)."""
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype not in dtypes:
+        raise ValueError("%s must be %s, got %s" % (name, " or ".join(map(str, dtypes)), t.dtype))
+    ok_shape = (t.dim() == 2 and t.shape[0] == shape[0] and
+                (t.shape[1] >= shape[1] if min_cols else t.shape[1] == shape[1]))
+    if not ok_shape or (t.numel() and t.stride(1) != 1):
+        raise ValueError("%s must be a row-major %s tensor, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def _check_bytes(t: torch.Tensor, nbytes: int, name: str):
+    if not t.is_cuda or t.dtype != torch.uint8 or not t.is_contiguous() or t.numel() < nbytes:
+        raise ValueError("%s must be a contiguous CUDA uint8 tensor of at least %d bytes" % (name, nbytes))
+
+
 def _require(t: torch.Tensor, dtype, name: str):
     if not t.is_cuda:
         raise ValueError("%s must be a CUDA tensor" % name)
@@ -85,6 +109,18 @@ def quant_act(x: torch.Tensor, layout: str = "both", out: QuantAct | None = None
         if flag & _lib.PURO_COLWISE:
             out.qt = torch.empty((cols, _round16(rows)), dtype=torch.uint8, device=dev)
             out.st = _blocked(cols, (rows + 127) // 128, dev)
+    else:
+        if (out.rows, out.cols) != (rows, cols):
+            raise ValueError("out was made for a [%d, %d] input" % (out.rows, out.cols))
+        if flag & _lib.PURO_ROWWISE:
+            _check_tensor(_need(out.q, "out has no row-wise codes"), (rows, cols), (torch.uint8,), "out.q")
+            _check_bytes(_need(out.s, "out has no row-wise scales"), blocked_scale_bytes(rows, cols // 128),
+                         "out.s")
+        if flag & _lib.PURO_COLWISE:
+            _check_tensor(_need(out.qt, "out has no transposed codes"), (cols, _round16(rows)),
+                          (torch.uint8,), "out.qt", min_cols=True)
+            _check_bytes(_need(out.st, "out has no transposed scales"),
+                         blocked_scale_bytes(cols, (rows + 127) // 128), "out.st")
     ptr = lambda t: t.data_ptr() if t is not None else None
     st = _lib.puro_fp8_quant_act(
         x.data_ptr(), rows, cols, x.stride(0), flag,
@@ -108,6 +144,17 @@ def quant_weight(w: torch.Tensor, transpose: bool = True, out: QuantWeight | Non
             torch.empty((k, n), dtype=torch.uint8, device=dev) if transpose else None,
             _blocked(n, k // 128, dev),
             _blocked(k, n // 128, dev) if transpose else None)
+    else:
+        if (out.n, out.k) != (n, k):
+            raise ValueError("out was made for a [%d, %d] weight" % (out.n, out.k))
+        _check_tensor(out.q, (n, k), (torch.uint8,), "out.q")
+        _check_bytes(out.s, (n // 128) * (k // 128), "out.s")
+        if out.s_fwd is not None:
+            _check_bytes(out.s_fwd, blocked_scale_bytes(n, k // 128), "out.s_fwd")
+        if out.qt is not None:
+            _check_tensor(out.qt, (k, n), (torch.uint8,), "out.qt", min_cols=True)
+            if out.s_bwd is not None:
+                _check_bytes(out.s_bwd, blocked_scale_bytes(k, n // 128), "out.s_bwd")
     ptr = lambda t: t.data_ptr() if t is not None else None
     st = _lib.puro_fp8_quant_weight(
         w.data_ptr(), n, k, w.stride(0), out.q.data_ptr(), out.q.stride(0), out.s.data_ptr(),
@@ -122,8 +169,11 @@ def gemm_fprop(xq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) -
     m, k, n = xq.rows, xq.cols, wq.n
     if wq.k != k:
         raise ValueError("inner dimensions differ: %d vs %d" % (k, wq.k))
+    _need(xq.q, "X was quantized without the row-wise layout fprop needs")
+    _need(wq.s_fwd, "the weight was quantized without its blocked fprop scales")
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=xq.q.device)
+    _check_tensor(out, (m, n), (torch.bfloat16,), "out", min_cols=False)
     st = _lib.puro_fp8_gemm_fprop(
         xq.q.data_ptr(), xq.q.stride(0), xq.s.data_ptr(),
         wq.q.data_ptr(), wq.q.stride(0), wq.s_fwd.data_ptr(),
@@ -139,8 +189,10 @@ def gemm_dgrad(dyq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) 
         raise ValueError("dY has %d columns, W has %d rows" % (n, wq.n))
     if wq.qt is None or wq.s_bwd is None:
         raise ValueError("dgrad needs the transposed weight codes (quant_weight(transpose=True))")
+    _need(dyq.q, "dY was quantized without the row-wise layout dgrad needs")
     if out is None:
         out = torch.empty((m, k), dtype=torch.bfloat16, device=dyq.q.device)
+    _check_tensor(out, (m, k), (torch.bfloat16,), "out")
     st = _lib.puro_fp8_gemm_dgrad(
         dyq.q.data_ptr(), dyq.q.stride(0), dyq.s.data_ptr(),
         wq.qt.data_ptr(), wq.qt.stride(0), wq.s_bwd.data_ptr(),
@@ -159,12 +211,13 @@ def gemm_wgrad(dyq: QuantAct, xq: QuantAct, out: torch.Tensor | None = None,
     m, n, k = dyq.rows, dyq.cols, xq.cols
     if xq.rows != m:
         raise ValueError("dY and X have different token counts")
+    _need(dyq.qt, "dY was quantized without the column-wise layout wgrad needs")
+    _need(xq.qt, "X was quantized without the column-wise layout wgrad needs")
     if out is None:
         if accumulate:
             raise ValueError("accumulate=True needs the FP32 buffer to add into")
         out = torch.empty((n, k), dtype=torch.bfloat16, device=dyq.qt.device)
-    if tuple(out.shape) != (n, k) or out.stride(1) != 1:
-        raise ValueError("out must be a row-major [n, k] tensor")
+    _check_tensor(out, (n, k), (torch.bfloat16, torch.float32), "out")
     if out.dtype == torch.float32:
         st = _lib.puro_fp8_gemm_wgrad_f32(
             dyq.qt.data_ptr(), dyq.qt.stride(0), dyq.st.data_ptr(),
@@ -190,8 +243,11 @@ def gemm_dgrad_wgrad(dyq: QuantAct, wq: QuantWeight, xq: QuantAct, dx: torch.Ten
     m, n, k = dyq.rows, dyq.cols, wq.k
     if wq.n != n or xq.rows != m or xq.cols != k:
         raise ValueError("shapes of dY, W and X do not agree")
-    if wq.qt is None:
+    if wq.qt is None or wq.s_bwd is None:
         raise ValueError("the weight was quantized without its transposed copy")
+    _need(dyq.q, "dY was quantized without the row-wise layout dgrad needs")
+    _need(dyq.qt, "dY was quantized without the column-wise layout wgrad needs")
+    _need(xq.qt, "X was quantized without the column-wise layout wgrad needs")
     dev = dyq.q.device
     if dx is None:
         dx = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
@@ -199,8 +255,8 @@ def gemm_dgrad_wgrad(dyq: QuantAct, wq: QuantWeight, xq: QuantAct, dx: torch.Ten
         if accumulate:
             raise ValueError("accumulate=True needs the FP32 buffer to add into")
         dw = torch.empty((n, k), dtype=torch.bfloat16, device=dev)
-    if tuple(dw.shape) != (n, k) or dw.stride(1) != 1 or tuple(dx.shape) != (m, k) or dx.stride(1) != 1:
-        raise ValueError("dx must be row-major [m, k] and dw row-major [n, k]")
+    _check_tensor(dx, (m, k), (torch.bfloat16,), "dx")
+    _check_tensor(dw, (n, k), (torch.bfloat16, torch.float32), "dw")
     if dw.dtype == torch.float32:
         kind = _lib.PURO_DW_F32_ACCUMULATE if accumulate else _lib.PURO_DW_F32
     elif dw.dtype == torch.bfloat16 and not accumulate:

@@ -169,3 +169,54 @@ def test_half_width_tail_tiles_match_whole_tiles(fp8, oracle_mod):
     rows = np.unique(np.linspace(0, m_split - 1, 24).astype(np.int64))
     assert_gemm_close(y_split[rows.tolist()], oracle_mod.linear_fprop(x[rows], w), oracle_mod,
                       "split-tail fprop")
+
+
+def test_wrapper_rejects_missing_layouts_and_bad_buffers(fp8):
+    """The torch-facing wrappers refuse, before any launch, a quantization
+    that lacks the layout an operation reads and an output buffer of the
+    wrong shape or type."""
+    x, w, dy = _layer(256, 256, 384, 21)
+    dev = torch.device("cuda")
+    x, w, dy = x.to(dev), w.to(dev), dy.to(dev)
+    x_row = fp8.quant_act(x, "rowwise")
+    x_col = fp8.quant_act(x, "colwise")
+    dy_row = fp8.quant_act(dy, "rowwise")
+    dy_both = fp8.quant_act(dy, "both")
+    wq = fp8.quant_weight(w)
+    wq_fwd = fp8.quant_weight(w, transpose=False)
+    with pytest.raises(ValueError):
+        fp8.gemm_fprop(x_col, wq)                               # no row-wise codes
+    with pytest.raises(ValueError):
+        fp8.gemm_fprop(x_row, wq, out=torch.empty(256, 128, dtype=torch.bfloat16, device=dev))
+    with pytest.raises(ValueError):
+        fp8.gemm_fprop(x_row, wq, out=torch.empty(256, 256, dtype=torch.float32, device=dev))
+    with pytest.raises(ValueError):
+        fp8.gemm_dgrad(dy_row, wq_fwd)                          # no transposed weight
+    with pytest.raises(ValueError):
+        fp8.gemm_dgrad(dy_row, wq, out=torch.empty(255, 384, dtype=torch.bfloat16, device=dev))
+    with pytest.raises(ValueError):
+        fp8.gemm_wgrad(dy_row, x_col)                           # dY lacks column-wise codes
+    with pytest.raises(ValueError):
+        fp8.gemm_wgrad(dy_both, x_col, out=torch.empty(384, 256, dtype=torch.float32, device=dev))
+    with pytest.raises(ValueError):
+        fp8.gemm_wgrad(dy_both, x_col, out=torch.empty(256, 384, dtype=torch.bfloat16, device=dev),
+                       accumulate=True)
+    with pytest.raises(ValueError):
+        fp8.gemm_dgrad_wgrad(dy_both, wq, x_row)                # X lacks column-wise codes
+    with pytest.raises(ValueError):
+        fp8.gemm_dgrad_wgrad(dy_both, wq, x_col, dx=torch.empty(256, 384, dtype=torch.float32, device=dev))
+    with pytest.raises(ValueError):
+        fp8.quant_act(x, "both", out=x_row)                     # reused result lacks the transposed layout
+    with pytest.raises(ValueError):
+        fp8.quant_act(x[:128].contiguous(), "rowwise", out=x_row)   # made for another shape
+    with pytest.raises(ValueError):
+        fp8.quant_weight(w[:128].contiguous(), out=wq)
+    # reusing a matching result works and gives the same codes
+    again = fp8.quant_act(x, "rowwise", out=fp8.QuantAct(256, 384, torch.empty_like(x_row.q),
+                                                          torch.empty_like(x_row.s)))
+    torch.cuda.synchronize()
+    assert torch.equal(again.q, x_row.q)
+    # only the scales of real groups are defined: bytes of the fourth (absent)
+    # group slot are left as they were
+    assert np.array_equal(gpu_rowwise(again)[1], gpu_rowwise(x_row)[1])
+    assert fp8.device_status() == 0

@@ -67,12 +67,6 @@ struct QuantParams {
   int32_t tiles_c, tiles;
 };
 
-// Byte offset of (row r, group g) in a blocked scale array whose rows hold
-// g4 = ceil(groups / 4) chunks of 512 bytes per 128-row block.
-__device__ __forceinline__ int64_t blocked_offset(int64_t r, int64_t g, int64_t g4) {
-  return ((r >> 7) * g4 + (g >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (g & 3);
-}
-
 // Scale exponent from the BF16 bits of a group's amax (sign already cleared).
 __device__ __forceinline__ int scale_exponent_from_bits(uint32_t a) {
   if (a == 0) return 0;
@@ -98,9 +92,19 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float2 x) {
 
 // Four values (pairs a, b) times 2^-e (s2) -> four E4M3 codes in one word,
 // a.x in the low byte.  The packed multiply is exact (a power of two,
-// subnormals kept), then one RNE saturating conversion per value.
+// subnormals kept), then one RNE saturating conversion per value; the two
+// 16-bit results are joined by a register move rather than shift-and-or
+// (measured: 8 fewer ALU instructions per 32 values on sm_100a).
 __device__ __forceinline__ uint32_t encode4(float2 a, float2 b, float2 s2) {
-  return cvt_e4m3x2(__fmul2_rn(a, s2)) | (cvt_e4m3x2(__fmul2_rn(b, s2)) << 16);
+  const float2 x = __fmul2_rn(a, s2), y = __fmul2_rn(b, s2);
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(x.x), "f"(x.y), "f"(y.x), "f"(y.y));
+  return r;
 }
 
 // The two BF16 of a packed word widened to FP32 (exact).
@@ -142,11 +146,16 @@ __device__ __forceinline__ uint2 encode_col8(const uint4 (&v)[8], int l, float2 
   return o;
 }
 
-// Column l of the thread's block as codes into its transposed-tile row `row`:
-// RPT codes at chunk i ^ (j * 8 / RPT) of RPT bytes.
+// Column l of the thread's block as codes into its transposed-tile row `row`.
+// 8 rows per thread: 8 codes at 8-byte chunk i ^ 2(j & 7), so that a 16-byte
+// unit holds two consecutive chunks in order (one plain 16-byte load per 16
+// rows on the way out) while the 32 stores of a warp still fill 16 distinct
+// chunk positions twice (two wavefronts, the minimum for 256 bytes).
+// 4 rows per thread: 4 codes at 4-byte slot i ^ 2j (conflict-free; the
+// readout swaps the 8-byte halves of odd column groups).
 __device__ __forceinline__ void put_col_codes(uint8_t* row, const uint4 (&v)[8], int l, float2 s2,
                                               int i, int j) {
-  *reinterpret_cast<uint2*>(row + ((i ^ j) << 3)) = encode_col8(v, l, s2);
+  *reinterpret_cast<uint2*>(row + ((i ^ (2 * (j & 7))) << 3)) = encode_col8(v, l, s2);
 }
 
 __device__ __forceinline__ void put_col_codes(uint8_t* row, const uint4 (&v)[4], int l, float2 s2,
@@ -161,16 +170,41 @@ __device__ __forceinline__ uint4 lds_v4(const uint8_t* p) {
   return *reinterpret_cast<const uint4*>(p);
 }
 
+// Row k's amax (BF16 bits) out of the row-pair words of row_amax, for a
+// lane-dependent k: byte permutes pick the half-word (a plain or selected
+// array index would be lowered to a local-memory round trip).
+template <int NQ>
+__device__ __forceinline__ uint32_t pick_row_amax(const uint32_t (&rm)[NQ], int k) {
+  static_assert(NQ == 2 || NQ == 4, "2 or 4 row-pair words");
+  const uint32_t b = 2u * static_cast<uint32_t>(k & 3);  // byte of the half within a word pair
+  const uint32_t sel = b | ((b + 1u) << 4);
+  uint32_t w = __byte_perm(rm[0], rm[1], sel);
+  if constexpr (NQ == 4) w = (k & 4) ? __byte_perm(rm[2], rm[3], sel) : w;
+  return w & 0xFFFFu;
+}
+
+// Byte offset, inside one 512-byte chunk of a blocked scale array, of the
+// chunk's row r (0..127).
+__device__ __forceinline__ uint32_t blocked_in_chunk(int r) {
+  return static_cast<uint32_t>((r & 31) * 16 + ((r >> 5) & 3) * 4);
+}
+
 // RSHFL selects how the row scales reach the threads (ROW without BLOCK):
 // one thread per row derives the exponent and the 16 threads of the row read
 // it with shuffles (fewer ALU instructions: faster when each CTA has only a
 // few tiles), or all 16 derive it themselves (no cross-lane latency on the
 // encode path: faster on long tile streams).  Both give identical results.
+//
+// Addressing is kept out of the per-element work: every output pointer is
+// formed once per tile from per-thread constants and advanced by its stride,
+// and the ragged-edge tests are one 32-bit compare against a per-tile count.
 template <bool ROW, bool COL, bool BLOCK, bool RSHFL>
 __global__ void __launch_bounds__(kQThreads, 2)
     quant_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantParams p) {
   constexpr uint32_t kMag = 0x7FFF7FFFu;
   constexpr int kWarps = kQThreads / 32;
+  constexpr int RPT = kQRpt;
+  constexpr int kColsPerPass = kQThreads / 8;  // transposed rows copied out per pass
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -182,7 +216,6 @@ __global__ void __launch_bounds__(kQThreads, 2)
   uint64_t* full = reinterpret_cast<uint64_t*>(blk_part + kWarps);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kQStages);
 
-  constexpr int RPT = kQRpt;
   const int tid = threadIdx.x;
   const int i = tid >> 4, j = tid & 15, warp = tid >> 5;
   // tiles t = blockIdx.x + it * gridDim.x, walked as (row tile, col tile)
@@ -214,6 +247,16 @@ __global__ void __launch_bounds__(kQThreads, 2)
   };
   if (tid == 0)
     while (p_it < my_tiles && p_it < kQStages) issue_next();
+
+  // per-thread constants of the output addressing
+  const uint32_t s_in_chunk = blocked_in_chunk(RPT * i + (j & (RPT - 1)));  // row scale byte (j < RPT)
+  const uint32_t st_in_chunk = blocked_in_chunk(2 * (tid & 63));            // column scale bytes (tid < 64)
+  const int c_base = tid >> 3, part = tid & 7;                               // transposed readout
+  const int64_t qt_pass_stride = (int64_t)kColsPerPass * p.ld_qt;
+  // 4 rows per thread: the readout's 16-byte unit has its 8-byte halves
+  // swapped for odd column groups, the same parity in every pass
+  // (kColsPerPass is a multiple of 16)
+  const bool swap_halves = RPT == 4 && ((c_base >> 3) & 1);
 
   int32_t tr = (int32_t)blockIdx.x / p.tiles_c, tc = (int32_t)blockIdx.x % p.tiles_c;
   for (int32_t it = 0; it < my_tiles; ++it) {
@@ -282,35 +325,38 @@ __global__ void __launch_bounds__(kQThreads, 2)
       if (tid == 0) p.sw[tr * p.tiles_c + tc] = static_cast<uint8_t>(e_blk + 127);
     }
 
-    // ---- in-place codes (ROW, BLOCK) and the row scale bytes.  Rows
-    // 8i..8i+7 share one 32-row group, so their scale bytes sit 16 apart.
+    // ---- in-place codes (ROW, BLOCK) and the row scale bytes; thread j < RPT
+    // owns the scale byte of row RPT*i + j
     if (ROW || BLOCK) {
-      uint8_t* qrow = p.q + (int64_t)(r0 + RPT * i) * p.ld_q + c0 + 8 * j;
+      uint8_t* qrow = p.q + (int64_t)(r0 + RPT * i) * p.ld_q + (c0 + 8 * j);
+      const int32_t nrow = (int32_t)(p.rows - r0) - RPT * i;  // rows of the block that exist
+      uint8_t* sbyte = BLOCK ? nullptr : p.s + ((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_in_chunk;
       if (RSHFL && !BLOCK) {
-        // thread j (< 8) of the 16 sharing rows 8i..8i+7 derives row 8i+j's
-        // exponent; the others read 2^-e from it with a shuffle
-        const int kk = j & (RPT - 1);
-        const uint32_t w = rowmax[kk >> 1];
-        const int e = scale_exponent_from_bits((kk & 1) ? (w >> 16) : (w & 0xFFFFu));
-        const float s_mine = pow2_neg_x2(e).x;
-        if (j < RPT) p.s[blocked_offset(r0 + RPT * i, tc, p.s_g4) + 16 * j] = static_cast<uint8_t>(e + 127);
+        // thread j derives row RPT*i + j's exponent; the 16 threads of the
+        // rows read 2^-e of row k from thread k
+        const int e_mine = scale_exponent_from_bits(pick_row_amax(rowmax, j & (RPT - 1)));
+        if (j < RPT) *sbyte = static_cast<uint8_t>(e_mine + 127);
+        const float s_mine = pow2_neg_x2(e_mine).x;
         const int lane16 = tid & 16;
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
           const float sk = __shfl_sync(0xFFFFFFFFu, s_mine, lane16 + k);
           const uint2 o = encode_row8(v[k], make_float2(sk, sk));
-          if (r0 + RPT * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
+          if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
+          qrow += p.ld_q;
         }
       } else {
-        // every thread derives the exponents of its 8 rows itself
-        uint8_t* srow = BLOCK ? nullptr : p.s + blocked_offset(r0 + RPT * i, tc, p.s_g4);
+        // every thread derives the exponents of its rows itself (the scale
+        // byte is stored inside the loop: deriving it ahead of the encodes was
+        // measured 10 % slower on long tile streams)
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
           const uint32_t m = (k & 1) ? (rowmax[k >> 1] >> 16) : (rowmax[k >> 1] & 0xFFFFu);
           const int e = BLOCK ? e_blk : scale_exponent_from_bits(m);
           const uint2 o = encode_row8(v[k], pow2_neg_x2(e));
-          if (r0 + RPT * i + k < p.rows) *reinterpret_cast<uint2*>(qrow + k * p.ld_q) = o;
-          if (!BLOCK && j == k) srow[16 * k] = static_cast<uint8_t>(e + 127);
+          if (!BLOCK && j == k) *sbyte = static_cast<uint8_t>(e + 127);
+          if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
+          qrow += p.ld_q;
         }
       }
     }
@@ -326,19 +372,16 @@ __global__ void __launch_bounds__(kQThreads, 2)
         __syncthreads();
         if (tid < 64) {
           // columns 2*tid and 2*tid+1: amax over the 8 warps, then the exponent,
-          // its scale byte (columns 8j..8j+7 sit 16 bytes apart in the blocked
-          // array) and 2^-e for every thread's encode
+          // its scale byte and 2^-e for every thread's encode
           uint32_t m = 0;
 #pragma unroll
           for (int w = 0; w < kWarps; ++w) m = __vmaxu2(m, col_part[(w * 16 + (tid >> 2)) * 4 + (tid & 3)]);
           const int e0 = scale_exponent_from_bits(m & 0xFFFFu);
           const int e1 = scale_exponent_from_bits(m >> 16);
-          const int c = 2 * tid;
-          uint8_t* scol = p.st + blocked_offset(c0 + (c & ~7), tr, p.st_g4) + 16 * (c & 7);
+          uint8_t* scol = p.st + ((int64_t)tc * p.st_g4 + (tr >> 2)) * 512 + (tr & 3) + st_in_chunk;
           scol[0] = static_cast<uint8_t>(e0 + 127);
           scol[16] = static_cast<uint8_t>(e1 + 127);
-          col_scale[c] = pow2_neg_x2(e0).x;
-          col_scale[c + 1] = pow2_neg_x2(e1).x;
+          *reinterpret_cast<float2*>(&col_scale[2 * tid]) = make_float2(pow2_neg_x2(e0).x, pow2_neg_x2(e1).x);
         }
         __syncthreads();
       }
@@ -352,28 +395,33 @@ __global__ void __launch_bounds__(kQThreads, 2)
 #pragma unroll
       for (int l = 0; l < 8; ++l) {
         const float2 s2 = BLOCK ? pow2_neg_x2(e_blk) : make_float2(cs[l], cs[l]);
-        // row (8j+l) of the transposed tile: this thread's RPT codes form chunk
-        // i ^ (j * 8 / RPT) of RPT bytes (the XOR spreads a warp's 16 j over
-        // distinct banks; the 16-byte readout below undoes it)
+        // row (8j+l) of the transposed tile: this thread's RPT codes go to an
+        // XOR-swizzled chunk (put_col_codes) that the readout below undoes
         put_col_codes(qt_s + (8 * j + l) * 128, v, l, s2, i, j);
       }
       __syncthreads();
+      // transposed row c = pass * kColsPerPass + c_base, rows 16*part.. of the
+      // tile: with jj = c / 8 its 16 codes sit in 16-byte unit part ^ (jj & 7)
+      // (8 rows per thread) or part ^ (jj >> 1) (4 rows per thread)
+      if (r0 + 16 * part < p.rows) {
+        uint8_t* dst = p.qt + (int64_t)(c0 + c_base) * p.ld_qt + (r0 + 16 * part);
 #pragma unroll
-      for (int pass = 0; pass < 1024 / kQThreads; ++pass) {
-        const int idx = pass * kQThreads + tid;
-        const int c = idx >> 3, part = idx & 7;
-        const int jj = (c >> 3) & 15;
-        const uint4 w = lds_v4(qt_s + c * 128 + ((part ^ (jj >> 1)) << 4));
-        const uint4 o = (jj & 1) ? make_uint4(w.z, w.w, w.x, w.y) : w;
-        const int32_t rr = r0 + 16 * part;
-        if (rr < p.rows) *reinterpret_cast<uint4*>(p.qt + (int64_t)(c0 + c) * p.ld_qt + rr) = o;
+        for (int pass = 0; pass < 128 / kColsPerPass; ++pass) {
+          const int c = pass * kColsPerPass + c_base;
+          const int unit = part ^ (RPT == 8 ? ((c >> 3) & 7) : ((c >> 4) & 7));
+          uint4 w = lds_v4(qt_s + c * 128 + (unit << 4));
+          if (swap_halves) w = make_uint4(w.z, w.w, w.x, w.y);
+          *reinterpret_cast<uint4*>(dst) = w;
+          dst += qt_pass_stride;
+        }
       }
     }
 
     if (BLOCK && tid < 128) {
       const uint8_t b = static_cast<uint8_t>(e_blk + 127);
-      if (p.sw_fwd) p.sw_fwd[blocked_offset(r0 + tid, tc, p.fwd_g4)] = b;
-      if (p.sw_bwd) p.sw_bwd[blocked_offset(c0 + tid, tr, p.bwd_g4)] = b;
+      const uint32_t in_chunk = blocked_in_chunk(tid);
+      if (p.sw_fwd) p.sw_fwd[((int64_t)tr * p.fwd_g4 + (tc >> 2)) * 512 + (tc & 3) + in_chunk] = b;
+      if (p.sw_bwd) p.sw_bwd[((int64_t)tc * p.bwd_g4 + (tr >> 2)) * 512 + (tr & 3) + in_chunk] = b;
     }
     if (COL || BLOCK) __syncthreads();  // shared tiles are reused by the next tile
     tc += tc_step;

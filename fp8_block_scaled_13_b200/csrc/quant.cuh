@@ -330,12 +330,12 @@ __global__ void __launch_bounds__(kQThreads, 2)
     if (ROW || BLOCK) {
       uint8_t* qrow = p.q + (int64_t)(r0 + RPT * i) * p.ld_q + (c0 + 8 * j);
       const int32_t nrow = (int32_t)(p.rows - r0) - RPT * i;  // rows of the block that exist
-      uint8_t* sbyte = BLOCK ? nullptr : p.s + ((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_in_chunk;
       if (RSHFL && !BLOCK) {
         // thread j derives row RPT*i + j's exponent; the 16 threads of the
         // rows read 2^-e of row k from thread k
         const int e_mine = scale_exponent_from_bits(pick_row_amax(rowmax, j & (RPT - 1)));
-        if (j < RPT) *sbyte = static_cast<uint8_t>(e_mine + 127);
+        if (j < RPT)
+          p.s[((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_in_chunk] = static_cast<uint8_t>(e_mine + 127);
         const float s_mine = pow2_neg_x2(e_mine).x;
         const int lane16 = tid & 16;
 #pragma unroll
@@ -347,14 +347,16 @@ __global__ void __launch_bounds__(kQThreads, 2)
         }
       } else {
         // every thread derives the exponents of its rows itself (the scale
-        // byte is stored inside the loop: deriving it ahead of the encodes was
-        // measured 10 % slower on long tile streams)
+        // byte is stored inside the loop, its address formed there: deriving
+        // the byte ahead of the encodes, or keeping its pointer live across
+        // the loop, was measured 10 % slower on long tile streams)
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
           const uint32_t m = (k & 1) ? (rowmax[k >> 1] >> 16) : (rowmax[k >> 1] & 0xFFFFu);
           const int e = BLOCK ? e_blk : scale_exponent_from_bits(m);
           const uint2 o = encode_row8(v[k], pow2_neg_x2(e));
-          if (!BLOCK && j == k) *sbyte = static_cast<uint8_t>(e + 127);
+          if (!BLOCK && j == k)
+            p.s[((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_in_chunk] = static_cast<uint8_t>(e + 127);
           if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
           qrow += p.ld_q;
         }
@@ -423,7 +425,9 @@ __global__ void __launch_bounds__(kQThreads, 2)
       if (p.sw_fwd) p.sw_fwd[((int64_t)tr * p.fwd_g4 + (tc >> 2)) * 512 + (tc & 3) + in_chunk] = b;
       if (p.sw_bwd) p.sw_bwd[((int64_t)tc * p.bwd_g4 + (tr >> 2)) * 512 + (tr & 3) + in_chunk] = b;
     }
-    if (COL || BLOCK) __syncthreads();  // shared tiles are reused by the next tile
+    // No barrier here: the shared tiles (qt_s, col_part, blk_part) are next
+    // written after the __syncthreads_or at the top of the next iteration,
+    // which no thread passes before every thread has finished this tile.
     tc += tc_step;
     tr += tr_step;
     if (tc >= p.tiles_c) { tc -= p.tiles_c; ++tr; }

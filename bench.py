@@ -317,7 +317,7 @@ def run_ours(args):
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(wl, dev, K=min(K, 10), warmup=2, accum=A)
+        e2e = run_e2e(wl, dev, K=min(K, 40), warmup=2, accum=A)
         if world > 1:
             t = torch.tensor([e2e["ms_per_step"]], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -538,11 +538,13 @@ def run_e2e(wl, dev, K, warmup, accum):
     """Same step through the public API with pinned host inputs/outputs, inside
     the timed region: every step copies X and dY in (and, at the start of each
     `accum`-step accumulation window, W, which is then quantized once for the
-    window), runs forward and backward (dW added into the FP32 main grads),
-    and copies Y, dX and the main grads back.  The copies are pipelined across
-    steps the way a training loop would: step i+1's inputs go up on a copy
-    stream while step i computes, and step i's results come down on another
-    while step i+1 computes (double-buffered buffers, ordered by events)."""
+    window), runs forward and backward (dW added into the FP32 main grads), and
+    copies Y and dX back; the main grads go back when they are complete, at
+    the end of each window (and of the run), as an optimizer would read them.
+    The copies are pipelined across steps the way a training loop would: step
+    i+1's inputs go up on a copy stream while step i computes, and step i's
+    results come down on another while step i+1 computes (double-buffered
+    inputs and outputs, ordered by events)."""
     import torch
     import fp8_block_scaled_13_b200 as fp8
     from fp8_block_scaled_13_b200.dp import MainGrads
@@ -551,24 +553,26 @@ def run_e2e(wl, dev, K, warmup, accum):
     host_w = [L.w.pin_memory() for L in wl.layers]
     host_in = [[(L.x.pin_memory(), L.dy.pin_memory()) for L in wl.layers] for _ in range(nbuf)]
     host_out = [[(torch.empty((L.m, L.n), dtype=torch.bfloat16).pin_memory(),
-                  torch.empty((L.m, L.k), dtype=torch.bfloat16).pin_memory(),
-                  torch.empty((L.n, L.k), dtype=torch.float32).pin_memory()) for L in wl.layers]
+                  torch.empty((L.m, L.k), dtype=torch.bfloat16).pin_memory()) for L in wl.layers]
                 for _ in range(nbuf)]
+    host_dw = [torch.empty((L.n, L.k), dtype=torch.float32).pin_memory() for L in wl.layers]
     dev_w = [torch.empty_like(w, device=dev) for w in host_w]
     dev_in = [[(torch.empty_like(x, device=dev), torch.empty_like(dy, device=dev))
                for (x, dy) in host_in[0]] for _ in range(nbuf)]
     wq = [None] * len(wl.layers)
     results = [None] * nbuf   # device outputs (Y, dX) of the step that used buffer b
-    grads = [MainGrads([(L.n, L.k) for L in wl.layers], device=dev) for _ in range(nbuf)]
+    grads = MainGrads([(L.n, L.k) for L in wl.layers], device=dev)
     bytes_w = sum(t.numel() * t.element_size() for t in host_w)
     bytes_in = sum(t.numel() * t.element_size() for tup in host_in[0] for t in tup)
-    d2h = sum(t.numel() * t.element_size() for tup in host_out[0] for t in tup)
+    bytes_out = sum(t.numel() * t.element_size() for tup in host_out[0] for t in tup)
+    bytes_dw = sum(t.numel() * t.element_size() for t in host_dw)
     comp = torch.cuda.current_stream()
     up = torch.cuda.Stream()
     down = torch.cuda.Stream()
     ev_up = [torch.cuda.Event() for _ in range(nbuf)]      # inputs of buffer b are on the device
     ev_done = [torch.cuda.Event() for _ in range(nbuf)]    # compute on buffer b finished
     ev_down = [torch.cuda.Event() for _ in range(nbuf)]    # results of buffer b are on the host
+    ev_dw_down = torch.cuda.Event()                        # the last window's dW is on the host
 
     def upload(i):
         b = i % nbuf
@@ -587,28 +591,34 @@ def run_e2e(wl, dev, K, warmup, accum):
         b = i % nbuf
         comp.wait_event(ev_up[b])
         comp.wait_event(ev_down[b])   # the previous results of buffer b went down
+        if i % accum == 0:
+            comp.wait_event(ev_dw_down)   # the previous window's dW went down
+            grads.zero_()
         outs = []
         for li, (x, dy) in enumerate(dev_in[b]):
             if i % accum == 0:
                 y, xq, wq[li] = fp8.linear_forward(x, dev_w[li])
             else:
                 y, xq, _ = fp8.linear_forward(x, wq=wq[li])
-            dx, _ = fp8.linear_backward(dy, xq, wq[li], main_grad=grads[b][li])
+            dx, _ = fp8.linear_backward(dy, xq, wq[li], main_grad=grads[li])
             y.record_stream(down)
             dx.record_stream(down)
             outs.append((y, dx))
         results[b] = outs
         ev_done[b].record(comp)
 
-    def download(i):
+    def download(i, last):
         b = i % nbuf
         with torch.cuda.stream(down):
             down.wait_event(ev_done[b])
-            for li, ((hy, hdx, hdw), (y, dx)) in enumerate(zip(host_out[b], results[b])):
+            for li, ((hy, hdx), (y, dx)) in enumerate(zip(host_out[b], results[b])):
                 hy.copy_(y, non_blocking=True)
                 hdx.copy_(dx, non_blocking=True)
-                hdw.copy_(grads[b][li], non_blocking=True)
             ev_down[b].record(down)
+            if i % accum == accum - 1 or last:
+                for hdw, g in zip(host_dw, grads.views):
+                    hdw.copy_(g, non_blocking=True)
+                ev_dw_down.record(down)
 
     def run(n):
         upload(0)
@@ -616,7 +626,7 @@ def run_e2e(wl, dev, K, warmup, accum):
             if i + 1 < n:
                 upload(i + 1)
             compute(i)
-            download(i)
+            download(i, i == n - 1)
         torch.cuda.synchronize()
 
     run(warmup)
@@ -629,7 +639,8 @@ def run_e2e(wl, dev, K, warmup, accum):
     torch.cuda.synchronize()
     windows = (K + accum - 1) // accum
     return {"ms_per_step": s.elapsed_time(e) / K,
-            "h2d": int(bytes_in + bytes_w * windows / K), "d2h": d2h}
+            "h2d": int(bytes_in + bytes_w * windows / K),
+            "d2h": int(bytes_out + bytes_dw * windows / K)}
 
 
 # ---------------------------------------------------------------- CPU oracle

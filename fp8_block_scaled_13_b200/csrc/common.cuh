@@ -179,6 +179,16 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
+// L2 prefetch of one tile through a tensor map (no shared memory, no
+// barrier): a hint that warms L2 ahead of the real load.  The x coordinate
+// obeys the same 16-byte rule as a tiled load.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // Tiled bulk tensor loads global -> this CTA's shared memory; the transferred
 // bytes are counted on the mbarrier at shared::cluster address `bar` (with
 // CG = 2 it may be the leader CTA's barrier).  Out-of-range elements read 0.

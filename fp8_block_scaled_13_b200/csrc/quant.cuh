@@ -230,6 +230,19 @@ __global__ void __launch_bounds__(kQThreads, 2)
     prefetch_tmap(&tm_x);
   }
   __syncthreads();
+  if (tid == 0) {
+    // Warm L2 with this CTA's first tiles while the kernel before this one is
+    // still finishing.  A prefetch only moves data into L2, the point of
+    // coherence, and the loads that fill shared memory still follow the
+    // dependency wait below, so a producer's later writes are what they read.
+    int32_t r = (int32_t)blockIdx.x / p.tiles_c, c = (int32_t)blockIdx.x % p.tiles_c;
+    for (int32_t t = 0; t < kQStages && t < my_tiles; ++t) {
+      tma_prefetch_l2_2d(&tm_x, c * 128, r * 128);
+      c += tc_step;
+      r += tr_step;
+      if (c >= p.tiles_c) { c -= p.tiles_c; ++r; }
+    }
+  }
   // the input may come from the kernel just before this one on the stream
   pdl_wait();
   pdl_trigger();

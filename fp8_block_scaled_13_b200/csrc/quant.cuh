@@ -263,6 +263,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
   // per-thread constants of the output addressing
   const uint32_t s_in_chunk = blocked_in_chunk(RPT * i + (j & (RPT - 1)));  // row scale byte (j < RPT)
+  const uint32_t s_half_chunk = blocked_in_chunk(RPT * i + (j >> 1));      // the same, row j >> 1
   const uint32_t st_in_chunk = blocked_in_chunk(2 * (tid & 63));            // column scale bytes (tid < 64)
   const int c_base = tid >> 3, part = tid & 7;                               // transposed readout
   const int64_t qt_pass_stride = (int64_t)kColsPerPass * p.ld_qt;
@@ -313,7 +314,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
         cm[3] = __vmaxu2(cm[3], a3);
       }
     }
-    if (ROW || BLOCK) {
+    // Row reductions over the 16 lanes of a row group.  On the shared-scale
+    // path with 8 rows per thread this is a reduce-scatter (rs_row below);
+    // elsewhere every lane needs every row's amax: a full butterfly.
+    constexpr bool kRowScatter = ROW && !BLOCK && RSHFL && RPT == 8;
+    if ((ROW || BLOCK) && !kRowScatter) {
 #pragma unroll
       for (int q = 0; q < RPT / 2; ++q) {
 #pragma unroll
@@ -343,7 +348,36 @@ __global__ void __launch_bounds__(kQThreads, 2)
     if (ROW || BLOCK) {
       uint8_t* qrow = p.q + (int64_t)(r0 + RPT * i) * p.ld_q + (c0 + 8 * j);
       const int32_t nrow = (int32_t)(p.rows - r0) - RPT * i;  // rows of the block that exist
-      if (RSHFL && !BLOCK) {
+      if (kRowScatter) {
+        // Reduce-scatter of the four row-pair words over the 16 lanes (lane
+        // bits b3 b2 b1 b0 = j): at distance 8 a lane keeps the pair of words
+        // for rows 4*b3.. and sends the other pair, at distance 4 it keeps the
+        // word for rows 4*b3 + 2*b2 + {0, 1}, then distances 2 and 1 finish
+        // that word.  Lane j then holds row j >> 1 in half b1 and derives its
+        // exponent; even lanes store the scale byte, and row k's 2^-e is read
+        // from lane 2k.
+        const bool b3 = (j >> 3) & 1, b2 = (j >> 2) & 1, b1 = (j >> 1) & 1;
+        uint32_t k0 = b3 ? rowmax[2] : rowmax[0], k1 = b3 ? rowmax[3] : rowmax[1];
+        const uint32_t s0 = b3 ? rowmax[0] : rowmax[2], s1 = b3 ? rowmax[1] : rowmax[3];
+        k0 = __vmaxu2(k0, __shfl_xor_sync(0xFFFFFFFFu, s0, 8));
+        k1 = __vmaxu2(k1, __shfl_xor_sync(0xFFFFFFFFu, s1, 8));
+        uint32_t w = b2 ? k1 : k0;
+        w = __vmaxu2(w, __shfl_xor_sync(0xFFFFFFFFu, b2 ? k0 : k1, 4));
+        w = __vmaxu2(w, __shfl_xor_sync(0xFFFFFFFFu, w, 2));
+        w = __vmaxu2(w, __shfl_xor_sync(0xFFFFFFFFu, w, 1));
+        const int e_mine = scale_exponent_from_bits(b1 ? (w >> 16) : (w & 0xFFFFu));
+        if ((j & 1) == 0)
+          p.s[((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_half_chunk] = static_cast<uint8_t>(e_mine + 127);
+        const float s_mine = pow2_neg_x2(e_mine).x;
+        const int lane16 = tid & 16;
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+          const float sk = __shfl_sync(0xFFFFFFFFu, s_mine, lane16 + 2 * k);
+          const uint2 o = encode_row8(v[k], make_float2(sk, sk));
+          if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
+          qrow += p.ld_q;
+        }
+      } else if (RSHFL && !BLOCK) {
         // thread j derives row RPT*i + j's exponent; the 16 threads of the
         // rows read 2^-e of row k from thread k
         const int e_mine = scale_exponent_from_bits(pick_row_amax(rowmax, j & (RPT - 1)));

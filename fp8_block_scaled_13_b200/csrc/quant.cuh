@@ -13,8 +13,9 @@
 // 128x128 tiles of the BF16 input; a TMA ring of kQStages 32 KB tile buffers
 // keeps the next tiles in flight while the current one is processed, and a
 // stage is handed back to the TMA as soon as every thread has copied its part
-// into registers.  Thread (i, j) = (tid/16, tid%16) holds rows 8i..8i+7 and
-// columns 8j..8j+7.  From those registers:
+// into registers (the first tiles are also prefetched into L2 before the
+// kernel waits on its predecessor).  Thread (i, j) = (tid/16, tid%16) holds
+// rows 8i..8i+7 and columns 8j..8j+7.  From those registers:
 //   ROW   : row amax by a 16-lane shuffle reduction; codes stored in place.
 //   COL   : column amax by a shuffle + shared-memory reduction over the 8
 //           warps; codes transposed through an XOR-swizzled 16 KB shared tile

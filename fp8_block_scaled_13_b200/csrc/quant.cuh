@@ -84,13 +84,6 @@ __device__ __forceinline__ float2 pow2_neg_x2(int e) {
   return make_float2(f, f);
 }
 
-// Two FP32 values -> two E4M3 codes (RNE, satfinite); x.x in the low byte.
-__device__ __forceinline__ uint32_t cvt_e4m3x2(float2 x) {
-  uint16_t c;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(x.y), "f"(x.x));
-  return c;
-}
-
 // Four values (pairs a, b) times 2^-e (s2) -> four E4M3 codes in one word,
 // a.x in the low byte.  The packed multiply is exact (a power of two,
 // subnormals kept), then one RNE saturating conversion per value; the two

@@ -12,6 +12,8 @@ Layouts (see include/puro_fp8.h):
 """
 from __future__ import annotations
 
+import dataclasses
+import functools
 from dataclasses import dataclass
 
 import torch
@@ -33,6 +35,35 @@ def _blocked(rows: int, groups: int, dev) -> torch.Tensor:
 
 def _stream() -> int:
     return torch.cuda.current_stream().cuda_stream
+
+
+def _tensors(obj):
+    if isinstance(obj, torch.Tensor):
+        yield obj
+    elif dataclasses.is_dataclass(obj) and not isinstance(obj, type):
+        for f in dataclasses.fields(obj):
+            v = getattr(obj, f.name)
+            if isinstance(v, torch.Tensor):
+                yield v
+
+
+def _on_operand_device(fn):
+    """Run a wrapper on the device its tensors live on.  The library launches
+    on the current CUDA device and takes the current stream, so operands on
+    another device are made current for the call; operands spread over
+    several devices are refused."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        devs = {t.device for a in (*args, *kwargs.values()) for t in _tensors(a)}
+        if len(devs) > 1:
+            raise ValueError("%s: operands are on different devices (%s)"
+                             % (fn.__name__, ", ".join(sorted(str(d) for d in devs))))
+        dev = devs.pop() if devs else None
+        if dev is not None and dev.type == "cuda":
+            with torch.cuda.device(dev):
+                return fn(*args, **kwargs)
+        return fn(*args, **kwargs)
+    return wrapper
 
 
 def _check(status: int, where: str):
@@ -95,6 +126,7 @@ class QuantWeight:
     s_bwd: torch.Tensor | None = None  # blocked: k rows x n/128 groups (dgrad B scales)
 
 
+@_on_operand_device
 def quant_act(x: torch.Tensor, layout: str = "both", out: QuantAct | None = None) -> QuantAct:
     """1x128 quantization of an activation/gradient x [rows, cols] (BF16)."""
     _require(x, torch.bfloat16, "x")
@@ -131,6 +163,7 @@ def quant_act(x: torch.Tensor, layout: str = "both", out: QuantAct | None = None
     return out
 
 
+@_on_operand_device
 def quant_weight(w: torch.Tensor, transpose: bool = True, out: QuantWeight | None = None) -> QuantWeight:
     """128x128 block quantization of a weight w [n, k] (BF16)."""
     _require(w, torch.bfloat16, "w")
@@ -164,6 +197,7 @@ def quant_weight(w: torch.Tensor, transpose: bool = True, out: QuantWeight | Non
     return out
 
 
+@_on_operand_device
 def gemm_fprop(xq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) -> torch.Tensor:
     """Y = X W^T [m, n] BF16 from the ROWWISE quantization of X and the weight's."""
     m, k, n = xq.rows, xq.cols, wq.n
@@ -182,6 +216,7 @@ def gemm_fprop(xq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) -
     return out
 
 
+@_on_operand_device
 def gemm_dgrad(dyq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) -> torch.Tensor:
     """dX = dY W [m, k] BF16 from the ROWWISE quantization of dY and W's transposed codes."""
     m, n, k = dyq.rows, dyq.cols, wq.k
@@ -201,6 +236,7 @@ def gemm_dgrad(dyq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) 
     return out
 
 
+@_on_operand_device
 def gemm_wgrad(dyq: QuantAct, xq: QuantAct, out: torch.Tensor | None = None,
                accumulate: bool = False) -> torch.Tensor:
     """dW = dY^T X [n, k] from the COLWISE quantizations of dY and X.
@@ -235,6 +271,7 @@ def gemm_wgrad(dyq: QuantAct, xq: QuantAct, out: torch.Tensor | None = None,
     return out
 
 
+@_on_operand_device
 def gemm_dgrad_wgrad(dyq: QuantAct, wq: QuantWeight, xq: QuantAct, dx: torch.Tensor | None = None,
                      dw: torch.Tensor | None = None, accumulate: bool = False):
     """dX = dY W and dW = dY^T X in one launch (tiles of both spread over the

@@ -59,7 +59,7 @@ def _on_operand_device(fn):
             raise ValueError("%s: operands are on different devices (%s)"
                              % (fn.__name__, ", ".join(sorted(str(d) for d in devs))))
         dev = devs.pop() if devs else None
-        if dev is not None and dev.type == "cuda":
+        if dev is not None and dev.type == "cuda" and dev.index != torch.cuda.current_device():
             with torch.cuda.device(dev):
                 return fn(*args, **kwargs)
         return fn(*args, **kwargs)

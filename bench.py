@@ -38,6 +38,10 @@ M_TOKENS = 8192
 # layer) from the ncu capture summarised in profiles/; None until captured
 # for the current kernel.
 GEMM_TRAFFIC_BYTES = 23338496 + 6511104  # QKV fprop launch, profiles/gemm_block_scaled_attn_proj_qkv_fprop.md
+# The same for one activation quantizer launch (quant_act BOTH of X [8192, 2048]);
+# its codes mostly stay in L2 for the GEMM that reads them next, so the DRAM
+# traffic is about half the algorithmic bytes (profiles/quant_kernel_attn_proj.md).
+QUANT_TRAFFIC_BYTES = 33584896 + 833536
 
 
 def _peaks():
@@ -390,6 +394,8 @@ def run_ours(args):
             "quantizers": {
                 "bound": "hbm", "achieved": round(quant_gbs, 1), "unit": "GB/s",
                 "peak": peaks["hbm_gbs"], "frac": round(quant_gbs / peaks["hbm_gbs"], 4),
+                "traffic": QUANT_TRAFFIC_BYTES,
+                "traffic_launch": "qkv.quant_x (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
             },
             "kernels": breakdown,
             "gpu_launches": launches_timed,

@@ -40,6 +40,7 @@ EXPORTS = (
     "puro_fp8_device_status",
     "puro_fp8_status_string",
     "puro_fp8_test_bounded_wait",
+    "puro_fp8_test_schedule",
 )
 
 _lib = None
@@ -76,6 +77,8 @@ def load() -> ctypes.CDLL:
     lib.puro_fp8_status_string.argtypes = [INT]
     lib.puro_fp8_status_string.restype = ctypes.c_char_p
     lib.puro_fp8_test_bounded_wait.argtypes = [I, P]
+    I32 = ctypes.c_int32
+    lib.puro_fp8_test_schedule.argtypes = [I32, I32, I32, I32, I32, P, P]
     for name in EXPORTS:
         if name not in ("puro_fp8_status_string", "puro_fp8_blocked_scale_bytes"):
             getattr(lib, name).restype = INT
@@ -137,3 +140,8 @@ def puro_fp8_status_string(status) -> str:
 
 def puro_fp8_test_bounded_wait(limit_ns, stream) -> int:
     return load().puro_fp8_test_bounded_wait(limit_ns, stream)
+
+
+def puro_fp8_test_schedule(units0, kblocks0, units1, kblocks1, clusters, offsets, units) -> int:
+    return load().puro_fp8_test_schedule(units0, kblocks0, units1, kblocks1, clusters, offsets,
+                                         units)

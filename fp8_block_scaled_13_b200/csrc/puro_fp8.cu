@@ -624,6 +624,30 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
 }
 }  // namespace puro
 
+extern "C" int puro_fp8_test_schedule(int32_t units0, int32_t kblocks0, int32_t units1,
+                                      int32_t kblocks1, int32_t clusters, int32_t* offsets,
+                                      int32_t* units) {
+  if (!offsets || !units) return PURO_ERR_NULL;
+  if (clusters < 1 || clusters > puro::kMaxSchedClusters || units0 < 0 || units1 < 0 ||
+      kblocks0 < 0 || kblocks1 < 0 || (int64_t)units0 + units1 > puro::kMaxSchedUnits)
+    return PURO_ERR_SHAPE;
+  static puro::GemmParams p;  // a few KB: kept off the caller's stack
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  memset(&p, 0, sizeof(p));
+  p.nprob = 2;
+  p.prob[0].kblocks = kblocks0;
+  p.prob[0].units = units0;
+  p.prob[1].kblocks = kblocks1;
+  p.prob[1].units = units1;
+  p.tiles0 = units0;
+  p.units = units0 + units1;
+  make_schedule(p, clusters);
+  for (int c = 0; c <= clusters; ++c) offsets[c] = p.sched_off[c];
+  for (int u = 0; u < p.units; ++u) units[u] = p.sched_unit[u];
+  return PURO_OK;
+}
+
 extern "C" int puro_fp8_test_bounded_wait(int64_t limit_ns, void* stream) {
   if (limit_ns < 1000) limit_ns = 1000;
   if (limit_ns > 5000000000ll) limit_ns = 5000000000ll;

@@ -245,6 +245,25 @@ PURO_API const char* puro_fp8_status_string(int status);
  */
 PURO_API int puro_fp8_test_bounded_wait(int64_t limit_ns, void* stream);
 
+/*
+ * puro_fp8_test_schedule -- host-only view of how a two-problem GEMM launch
+ * (puro_fp8_gemm_dgrad_wgrad) spreads its work units over the launch's
+ * clusters.  Problem 0 has `units0` units of `kblocks0` K blocks each, problem
+ * 1 `units1` units of `kblocks1`; units [0, units0) are problem 0's.  The
+ * units are taken longest first (cost = K blocks + 2, ties in unit order) and
+ * each goes to the least-loaded cluster so far (ties: lowest cluster index).
+ * On return cluster c runs units[offsets[c] .. offsets[c + 1]) in that order.
+ *   offsets : host array of clusters + 1 entries (written)
+ *   units   : host array of units0 + units1 entries (written)
+ * No device work.  PURO_ERR_NULL for a null array; PURO_ERR_SHAPE unless
+ * 1 <= clusters <= 128, units0, units1, kblocks0, kblocks1 >= 0 and
+ * units0 + units1 <= 2048 (the launch schedules at most that many units and
+ * falls back to round robin beyond).
+ */
+PURO_API int puro_fp8_test_schedule(int32_t units0, int32_t kblocks0, int32_t units1,
+                                    int32_t kblocks1, int32_t clusters, int32_t* offsets,
+                                    int32_t* units);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,7 +22,7 @@
  *     the three GEMMs (forward, data-gradient, weight-gradient) use blockwise
  *     E4M3; hidden flow stays BF16.
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent:
  *   - E4M3 is the OCP "FN" variant: bias 7, max finite 448, NaN 0x7F/0xFF,
  *     no infinities, subnormals 2^-6 * m/8.
  *   - The scale 2^e of a group is the smallest power of two with

@@ -34,13 +34,13 @@ METRIC = "FP8 block-scaled GEMM TFLOP/s (fprop/dgrad/wgrad) and % of B200 FP8 pe
 WORKLOAD = "attn_proj_m8192_h2048_qkv3072_o2048"
 SEED = 1
 M_TOKENS = 8192
-# dram__bytes_read.sum + dram__bytes_write.sum of one GEMM launch (fprop, QKV
-# layer) from the ncu capture summarised in profiles/; None until captured
-# for the current kernel.
-GEMM_TRAFFIC_BYTES = 23338496 + 6511104  # QKV fprop launch, profiles/gemm_block_scaled_attn_proj_qkv_fprop.md
+# dram__bytes_read.sum + dram__bytes_write.sum of one GEMM launch (the QKV
+# layer's fprop, 8192 x 3072 x 2048) from an ncu capture of this step; to be
+# set to None when the GEMM kernel changes until it is captured again.
+GEMM_TRAFFIC_BYTES = 23338496 + 6511104
 # The same for one activation quantizer launch (quant_act BOTH of X [8192, 2048]);
 # its codes mostly stay in L2 for the GEMM that reads them next, so the DRAM
-# traffic is about half the algorithmic bytes (profiles/quant_kernel_attn_proj.md).
+# traffic is about half the algorithmic bytes.
 QUANT_TRAFFIC_BYTES = 33584896 + 833536
 
 

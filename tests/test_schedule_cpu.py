@@ -66,3 +66,15 @@ def test_schedule_argument_errors(lib):
     assert f(4, 1, 4, 1, 129, off.ctypes.data, units.ctypes.data) == -3
     assert f(2048, 1, 1, 1, 8, off.ctypes.data, units.ctypes.data) == -3
     assert f(-1, 1, 4, 1, 8, off.ctypes.data, units.ctypes.data) == -3
+
+
+def test_schedule_invariants_random(lib):
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=300, deadline=None)
+    @given(u0=st.integers(0, 1024), k0=st.integers(0, 200), u1=st.integers(0, 1024),
+           k1=st.integers(0, 200), clusters=st.integers(1, 128))
+    def check(u0, k0, u1, k1, clusters):
+        test_schedule_invariants(lib, u0, k0, u1, k1, clusters)
+
+    check()

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <functional>
@@ -140,13 +141,14 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, in
     return PURO_ERR_CUDA;
   auto kern = puro::quant_kernel<ROW, COL, BLOCK, RSHFL>;
   constexpr uint32_t smem = puro::quant_smem_bytes();
-  static bool attr_done[kMaxDevices] = {};
+  // per device, once (threads racing on the first call both set the same value)
+  static std::atomic<bool> attr_done[kMaxDevices] = {};
   int dev_id = 0;
   cudaGetDevice(&dev_id);
-  if (!attr_done[dev_id]) {
+  if (!attr_done[dev_id].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return PURO_ERR_CUDA;
-    attr_done[dev_id] = true;
+    attr_done[dev_id].store(true, std::memory_order_release);
   }
   const int64_t grid = p.tiles < 2 * (int64_t)sms ? p.tiles : 2 * (int64_t)sms;
   cudaLaunchConfig_t cfg = {};
@@ -256,7 +258,8 @@ int launch_gemm_cfg(const GemmArgs& g0, const GemmArgs* g1, DeviceInfo* dev, cud
     memcpy(m1, m0, sizeof(m0));  // unused by a one-problem launch
   }
   auto kern = puro::gemm_block_scaled_kernel<CG, BN, BK, OUT0, OUT1>;
-  static int max_clusters[kMaxDevices] = {};
+  // per device, once (threads racing on the first call both store the same value)
+  static std::atomic<int> max_clusters[kMaxDevices] = {};
   int dev_id = 0;
   cudaGetDevice(&dev_id);
   cudaLaunchConfig_t cfg = {};
@@ -272,14 +275,15 @@ int launch_gemm_cfg(const GemmArgs& g0, const GemmArgs* g1, DeviceInfo* dev, cud
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;  // the occupancy query below uses the cluster attribute only
-  if (max_clusters[dev_id] == 0) {
+  if (max_clusters[dev_id].load(std::memory_order_acquire) == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
       return PURO_ERR_CUDA;
     int n = 0;
     cfg.gridDim = dim3(CG * (dev->sms / CG));
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = dev->sms / CG;
-    max_clusters[dev_id] = n < puro::kMaxSchedClusters ? n : puro::kMaxSchedClusters;
+    max_clusters[dev_id].store(n < puro::kMaxSchedClusters ? n : puro::kMaxSchedClusters,
+                               std::memory_order_release);
   }
   static thread_local puro::GemmParams p;  // ~4.5 KB: kept off the stack
   memset(&p, 0, sizeof(p));
@@ -293,7 +297,7 @@ int launch_gemm_cfg(const GemmArgs& g0, const GemmArgs* g1, DeviceInfo* dev, cud
     p.prob[i].tiles_m = (int32_t)((g.rows_a + C::kBM - 1) / C::kBM);
     p.prob[i].tiles_n = (int32_t)((g.rows_b + BN - 1) / BN);
   }
-  const int C_max = max_clusters[dev_id];
+  const int C_max = max_clusters[dev_id].load(std::memory_order_acquire);
   for (int i = 0; i < p.nprob; ++i) {
     const int64_t t = (int64_t)p.prob[i].tiles_m * p.prob[i].tiles_n;
     p.prob[i].split_from = (int32_t)t;

@@ -21,6 +21,11 @@
  *    puro_fp8_device_status().
  *  - Errors are returned as puro_status codes; nothing throws or aborts.  An
  *    argument error is detected on the host and returns before any launch.
+ *  - Calls work on the calling thread's current CUDA device.  Several host
+ *    threads may call the library at once (each with its own stream): the
+ *    per-device state (device checks, kernel attributes, launch limits) is
+ *    set up once behind a mutex or atomics, and launch parameters are
+ *    per-thread.
  *  - Element formats:
  *      BF16   : IEEE binary32 upper half (torch.bfloat16).
  *      E4M3   : OCP FP8 "FN" (torch.float8_e4m3fn): bias 7, max 448, NaN 0x7F

@@ -1,8 +1,7 @@
 """Benchmark of the block-scaled FP8 linear layer hot path on B200.
 
-One step = one micro-batch of the attention-projection workload (M = 8192
-tokens, hidden 2048; the fused QKV projection 2048->3072 and the output
-projection 2048->2048), for each of the two layers:
+A step is one forward + backward pass of every linear layer of a workload over
+one batch of M tokens (inputs resident in HBM).  For each layer:
   quant_act(X, both), fprop, quant_act(dY, both), and one launch computing
   dgrad and wgrad (dW added into FP32 main grads); quant_weight(W) (+
   transposed codes) runs once per gradient-accumulation window of --accum
@@ -10,16 +9,27 @@ projection 2048->2048), for each of the two layers:
 value = GEMM FLOPs of the step (2*M*N*K per GEMM, three GEMMs per layer)
 divided by the device time of the whole step (quantizers included).
 
-Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--accum A]
-                       [--impl ours|reference]
-With N > 1 (torchrun) every rank runs its own batch (data parallel, weak
-scaling) and every A steps the ranks all-reduce the FP32 weight gradients.
+The default workload is the full hidden-2048 / FFN-6144 transformer block
+(QKV 2048->3072, O 2048->2048, gate+up 2048->12288, down 6144->2048) at
+M = 32768 tokens, the largest single-GPU configuration; a sweep of the other
+configurations (attention projections, SwiGLU gate+up, heavy-tailed MLP down,
+the full block at M = 4096, 8000, 16384) follows as summaries in the same
+JSON line.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                       [--tokens M] [--accum A] [--impl ours|reference]
+                       [--no-sweep] [--no-e2e] [--no-cpu-baseline] [--no-bf16]
+                       [--no-ceiling]
+N > 1: every rank runs its own batch (data parallel, weak scaling) and every A
+steps the ranks all-reduce the FP32 weight gradients (NCCL).  Launched without
+torchrun, bench.py starts the N ranks itself (torch.distributed.run).
 """
 from __future__ import annotations
 
 import argparse
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -31,17 +41,30 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "FP8 block-scaled GEMM TFLOP/s (fprop/dgrad/wgrad) and % of B200 FP8 peak"
-WORKLOAD = "attn_proj_m8192_h2048_qkv3072_o2048"
-SEED = 1
-M_TOKENS = 8192
-# dram__bytes_read.sum + dram__bytes_write.sum of one GEMM launch (the QKV
-# layer's fprop, 8192 x 3072 x 2048) from an ncu capture of this step; to be
-# set to None when the GEMM kernel changes until it is captured again.
-GEMM_TRAFFIC_BYTES = 23338496 + 6511104
-# The same for one activation quantizer launch (quant_act BOTH of X [8192, 2048]);
-# its codes mostly stay in L2 for the GEMM that reads them next, so the DRAM
-# traffic is about half the algorithmic bytes.
-QUANT_TRAFFIC_BYTES = 33584896 + 833536
+
+# workload -> (default tokens, seed, shapes for the config record)
+WORKLOADS = {
+    "full_block": (32768, 4, "hidden 2048, FFN 6144: QKV 2048->3072, O 2048->2048, "
+                             "gate+up 2048->12288, down 6144->2048"),
+    "attn_proj": (8192, 1, "hidden 2048: QKV 2048->3072, O 2048->2048 (shared X)"),
+    "swiglu_gate_up": (16384, 2, "gate+up 2048->12288, 8 channels of X x50"),
+    "mlp_down_heavy": (16384, 3, "down 6144->2048, Student-t(3) X, Laplace dY, zero groups"),
+}
+SWEEP = [("attn_proj", 8192), ("swiglu_gate_up", 16384), ("mlp_down_heavy", 16384),
+         ("full_block", 4096), ("full_block", 8000), ("full_block", 16384)]
+# tokens per gradient-accumulation window: the pages' 1536 sequences /
+# (DP 12 x MBS 2) = 64 micro-batches of 2 x 4096 tokens
+WINDOW_TOKENS = 64 * 8192
+L2_BYTES = 126 * 1024 * 1024
+SPEC_FP8_TFLOPS = 4500.0     # B200 dense FP8 tensor-core peak (spec)
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch, from ncu captures
+# (one-pass metrics on the full-size default workload), keyed by launch name;
+# None when the kernel has changed since it was captured.
+GEMM_TRAFFIC_BYTES = None
+QUANT_TRAFFIC_BYTES = None
 
 
 def _peaks():
@@ -50,45 +73,70 @@ def _peaks():
         with open(path) as f:
             d = json.load(f)
         return d, "measured"
-    except OSError:
+    except (OSError, ValueError):
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def _parse_args():
+def _parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="full_block")
+    ap.add_argument("--tokens", dest="m", type=int, default=None,
+                    help="tokens per GPU per step (M)")
+    ap.add_argument("--accum", type=int, default=None,
+                    help="steps per gradient exchange (default: a window of 64 x 8192 tokens)")
+    ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-ceiling", action="store_true")
     ap.add_argument("--no-bf16", action="store_true")
-    ap.add_argument("--accum", type=int, default=64,
-                    help="micro-batch steps per gradient exchange (the pages: 1536 sequences / "
-                         "(DP 12 x MBS 2) = 64)")
-    return ap.parse_args()
+    args = ap.parse_args(argv)
+    if args.m is None:
+        args.m = WORKLOADS[args.workload][0]
+    if args.accum is None:
+        args.accum = max(1, WINDOW_TOKENS // args.m)
+    if args.gpus < 1 or args.steps < 1 or args.warmup < 0 or args.m < 1:
+        ap.error("--gpus, --steps, --tokens must be >= 1 and --warmup >= 0")
+    return args
+
+
+def make_workload(name: str, m: int, seed_offset: int = 0):
+    from fp8_block_scaled_13_b200 import inputs
+    seed = WORKLOADS[name][1] + seed_offset
+    return inputs.WORKLOADS[name](seed=seed, m=m)
+
+
+def workload_tag(name: str, m: int) -> str:
+    return "%s_m%d" % (name, m)
 
 
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    """nvidia-smi samples of the SM clock, utilisation and throttle reasons
+    while the context is open; the summary takes the median clock over the
+    samples taken under load (utilisation >= 50 %)."""
+
+    def __init__(self, gpu: str, period_ms: int = 50):
+        self.gpu = gpu
+        self.period = period_ms
         self.proc = None
         self.path = None
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
         os.close(fd)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         self.out = open(self.path, "w")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + q,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.period)],
                 stdout=self.out, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -117,31 +165,61 @@ class ClockSampler:
                 if len(parts) >= 9:
                     rows.append(parts)
         os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        return summarize_clocks(rows)
+
+
+def smi_id(device_index: int) -> str:
+    """nvidia-smi's name for a CUDA device: its UUID (device indexes differ
+    between CUDA and nvidia-smi when CUDA_VISIBLE_DEVICES is set)."""
+    try:
+        import torch
+        u = str(torch.cuda.get_device_properties(device_index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:  # noqa: BLE001  (older torch without a uuid field)
+        return str(device_index)
+
+
+def _num(s):
+    try:
+        return float(s)
+    except ValueError:
+        return None
+
+
+def summarize_clocks(rows):
+    """rows: nvidia-smi fields index, clocks.sm, clocks.max.sm, power.draw,
+    utilization.gpu, hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown,
+    sw_power_cap.  Median SM clock over the loaded samples (all samples if
+    none is loaded); every throttle reason seen Active in a loaded sample."""
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+    loaded = [r for r in rows if (_num(r[4]) or 0.0) >= 50.0]
+    use = loaded or rows
+    sm = [v for v in (_num(r[1]) for r in use) if v is not None]
+    mx = [v for v in (_num(r[2]) for r in rows) if v is not None]
+    pw = [v for v in (_num(r[3]) for r in use) if v is not None]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in use for i in range(4) if r[5 + i] == "Active"})
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(mx) if mx else None,
+            "power_w": round(statistics.median(pw), 1) if pw else None,
+            "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded)}
 
 
 # ---------------------------------------------------------------- our arm
 
 class Step:
-    """Device buffers of one step and the launch sequence, with an event pair
-    around every launch (on the launching stream)."""
+    """Device buffers of one step and the launch sequence, with an optional
+    event pair around every launch (on the launching stream)."""
 
-    def __init__(self, wl, dev, n_sets=3):
+    def __init__(self, wl, dev, n_sets):
         import torch
         import fp8_block_scaled_13_b200 as fp8
         from fp8_block_scaled_13_b200.dp import MainGrads
         self.fp8 = fp8
         self.torch = torch
         self.layers = wl.layers
-        # rotating input sets: each set is larger than L2 in total
+        # input sets: rotated so that every step's inputs come from HBM
         self.sets = []
         for _ in range(n_sets):
             self.sets.append([(L.x.to(dev), L.w.to(dev), L.dy.to(dev)) for L in wl.layers])
@@ -154,7 +232,7 @@ class Step:
             y = torch.empty((x.shape[0], w.shape[0]), dtype=torch.bfloat16, device=dev)
             dx = torch.empty_like(x)
             self.out.append((xq, wq, dyq, y, dx))
-        # FP32 weight gradients of both layers in one buffer: every step adds
+        # FP32 weight gradients of all layers in one buffer: every step adds
         # its dW into it (one micro-batch of gradient accumulation)
         self.grads = MainGrads([(w.shape[0], w.shape[1]) for (_, w, _) in self.sets[0]], device=dev)
         torch.cuda.synchronize()
@@ -170,9 +248,9 @@ class Step:
         return names
 
     def run(self, set_idx, events=None, weights=True):
-        """One micro-batch step.  The weights are quantized only when `weights`:
-        within a gradient-accumulation window they do not change, so the first
-        step's codes serve the whole window."""
+        """One step.  The weights are quantized only when `weights`: within a
+        gradient-accumulation window they do not change, so the first step's
+        codes serve the whole window."""
         fp8 = self.fp8
         ev = iter(events) if events is not None else None
 
@@ -197,6 +275,18 @@ class Step:
         self.grads.zero_()
 
 
+def input_set_bytes(wl) -> int:
+    return sum(t.numel() * t.element_size() for L in wl.layers for t in (L.x, L.w, L.dy))
+
+
+def n_input_sets(wl) -> int:
+    """Enough rotating input sets that the inputs a step reads were last read
+    at least three L2 capacities of traffic ago (one set when a single set
+    already is)."""
+    per = input_set_bytes(wl)
+    return max(1, min(3, -(-3 * L2_BYTES // per)))
+
+
 def _unit_costs(wl):
     """Algorithmic work per launch: FLOPs for the GEMMs, bytes for quantizers."""
     costs = {}
@@ -210,26 +300,18 @@ def _unit_costs(wl):
     return costs
 
 
-def run_ours(args):
+def measure(wl, dev, world, K, warmup, accum, gpu, inst_steps=100):
+    """Times K steps of the workload on the device (CUDA graphs of `accum`
+    steps, the gradient exchange between them) and, separately, per-launch
+    times from an instrumented replay.  Returns the raw measurements."""
     import torch
     import torch.distributed as dist
-    from fp8_block_scaled_13_b200 import inputs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-
-    wl = inputs.attn_proj(seed=SEED + rank, m=M_TOKENS)
-    step = Step(wl, dev)
-    costs = _unit_costs(wl)
-    gemm_flops = wl.gemm_flops()
-    A = max(1, min(args.accum, args.steps))
-    for i in range(args.warmup):
-        step.run(i % len(step.sets), weights=(i % A == 0))
+    n_sets = n_input_sets(wl)
+    step = Step(wl, dev, n_sets)
+    A = max(1, min(accum, K))
+    for i in range(warmup):
+        step.run(i % n_sets, weights=(i % A == 0))
     torch.cuda.synchronize()
     status = step.fp8.device_status()
     if status != 0:
@@ -237,17 +319,15 @@ def run_ours(args):
 
     # The timed steps run as CUDA graphs (kernel arguments, including the TMA
     # descriptors, are baked in), so the timed region holds device work only:
-    # a graph of `accum` micro-batch steps is replayed, and after each window
-    # the FP32 weight gradients are exchanged across the ranks (NCCL
-    # all-reduce, outside the graph) and cleared; exactly K steps in all (a
-    # shorter graph covers the remainder).  A separate graph with an event
-    # pair around every launch gives the per-kernel breakdown; it is replayed
-    # on its own because event nodes between kernels also cut the
-    # programmatic (PDL) edges that let a kernel's prologue overlap its
-    # predecessor's tail.
-    K = args.steps
+    # a graph of `accum` steps is replayed, and after each window the FP32
+    # weight gradients are exchanged across the ranks (NCCL all-reduce,
+    # outside the graph) and cleared; exactly K steps in all (a shorter graph
+    # covers the remainder).  A separate graph with an event pair around every
+    # launch gives the per-kernel breakdown; it is replayed on its own because
+    # event nodes between kernels also cut the programmatic (PDL) edges that
+    # let a kernel's prologue overlap its predecessor's tail.
     windows = [A] * (K // A) + ([K % A] if K % A else [])
-    K_inst = min(K, 100)
+    K_inst = min(K, inst_steps)
     inst_names = [step.launch_names(i % A == 0) for i in range(K_inst)]
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * len(nm))]
           for nm in inst_names]
@@ -260,10 +340,10 @@ def run_ours(args):
             graphs[n] = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graphs[n], stream=cap_stream):
                 for i in range(n):
-                    step.run(i % len(step.sets), weights=(i == 0))
+                    step.run(i % n_sets, weights=(i == 0))
         with torch.cuda.graph(graph_inst, stream=cap_stream):
             for i in range(K_inst):
-                step.run(i % len(step.sets), ev[i], weights=(i % A == 0))
+                step.run(i % n_sets, ev[i], weights=(i % A == 0))
     torch.cuda.synchronize()
     for g in graphs.values():  # untimed first replays of the instantiated graphs
         g.replay()
@@ -275,22 +355,21 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(gpu) as clk:
         t_start.record()
         for n in windows:
             graphs[n].replay()
             step.sync_grads(world)
         t_end.record()
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    graph_inst.replay()
-    torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        graph_inst.replay()
+        torch.cuda.synchronize()
     status = step.fp8.device_status()
     if status != 0:
         raise RuntimeError("device status %d in the timed region" % status)
-    clocks = clk.summary()
 
     total_ms = t_start.elapsed_time(t_end)
     per_launch = {name: [] for name in step.all_names}
@@ -304,27 +383,100 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_per_step = float(t.item())
     del graphs, graph_inst
+    return {"step": step, "ms_per_step": ms_per_step, "total_ms": total_ms, "accum": A,
+            "per_launch": per_launch, "clocks": clk.summary(), "launches_timed": launches_timed,
+            "inst_steps": K_inst, "n_sets": n_sets}
 
-    peaks, peak_kind = _peaks()
-    fp8_peak_tf = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    value = gemm_flops * world / (ms_per_step * 1e-3) / 1e12
 
-    gemm_ms = sum(statistics.mean(per_launch[n]) for n in step.all_names if costs[n][0] == "flops")
+def summarize(wl, res, peaks, peak_kind, world):
+    """value, GEMM roofline, quantizer roofline and per-kernel breakdown."""
+    costs = _unit_costs(wl)
+    gemm_flops = wl.gemm_flops()
+    names = res["step"].all_names
+    pl = res["per_launch"]
+    value = gemm_flops * world / (res["ms_per_step"] * 1e-3) / 1e12
+    gemm_ms = sum(statistics.mean(pl[n]) for n in names if costs[n][0] == "flops")
     gemm_tf = gemm_flops / (gemm_ms * 1e-3) / 1e12
     # quantizer bandwidth over every quantizer launch of the instrumented replay
-    quant_ms = sum(sum(per_launch[n]) for n in step.all_names if costs[n][0] == "bytes")
-    quant_bytes = sum(costs[n][1] * len(per_launch[n]) for n in step.all_names if costs[n][0] == "bytes")
+    quant_ms = sum(sum(pl[n]) for n in names if costs[n][0] == "bytes")
+    quant_bytes = sum(costs[n][1] * len(pl[n]) for n in names if costs[n][0] == "bytes")
     quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    act_names = [n for n in names if costs[n][0] == "bytes" and not n.endswith("quant_weight")]
+    act_ms = sum(sum(pl[n]) for n in act_names)
+    act_gbs = sum(costs[n][1] * len(pl[n]) for n in act_names) / (act_ms * 1e-3) / 1e9
     breakdown = {}
-    for n in step.all_names:
+    for n in names:
         kind, amount = costs[n]
-        ms = statistics.mean(per_launch[n])
+        ms = statistics.mean(pl[n])
         rate = amount / (ms * 1e-3) / (1e12 if kind == "flops" else 1e9)
         breakdown[n] = {"ms": round(ms, 5), ("tflops" if kind == "flops" else "gbs"): round(rate, 1)}
+    burst = 2.0 * peaks["bf16_tflops"]
+    sustained = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    per_step_ms = {"gemm": gemm_ms,
+                   "quant_act": act_ms / res["inst_steps"],
+                   "quant_weight": (quant_ms - act_ms) / res["inst_steps"]}
+    roofline = {
+        "bound": "tensor",
+        "kernel": "gemm_block_scaled_kernel (every GEMM launch of the step, FLOP-weighted)",
+        "achieved": round(gemm_tf, 1),
+        "peak": round(burst, 1),
+        "unit": "TFLOP/s",
+        "frac": round(gemm_tf / burst, 4),
+        "peak_source": "%s: 2 x bf16_tflops (burst cuBLAS BF16 GEMM) x the nominal FP8:BF16 "
+                       "ratio of 2; of %s" % (peak_kind, peak_kind),
+        "frac_vs_spec": round(gemm_tf / SPEC_FP8_TFLOPS, 4),
+        "spec_peak": SPEC_FP8_TFLOPS,
+        "frac_vs_sustained": round(gemm_tf / sustained, 4),
+        "sustained_peak": round(sustained, 1),
+        "traffic": GEMM_TRAFFIC_BYTES,
+    }
+    quant = {
+        "bound": "hbm", "achieved": round(quant_gbs, 1), "unit": "GB/s",
+        "peak": peaks["hbm_gbs"], "frac": round(quant_gbs / peaks["hbm_gbs"], 4),
+        "peak_source": "%s: hbm_gbs (STREAM-style copy); of %s" % (peak_kind, peak_kind),
+        "frac_vs_spec": round(quant_gbs / SPEC_HBM_GBS, 4), "spec_peak": SPEC_HBM_GBS,
+        "activations_only": {"achieved": round(act_gbs, 1),
+                             "frac": round(act_gbs / peaks["hbm_gbs"], 4)},
+        "traffic": QUANT_TRAFFIC_BYTES,
+        "what": "every quantizer launch of the instrumented replay, algorithmic bytes over "
+                "per-launch event time (each launch timed on its own, without the overlap "
+                "with its neighbours that the timed graphs have)",
+    }
+    return {"value": value, "gemm_tf": gemm_tf, "roofline": roofline, "quantizers": quant,
+            "kernels": breakdown, "gemm_flops": gemm_flops,
+            "time_split_ms_per_step": {k: round(v, 4) for k, v in per_step_ms.items()},
+            "pct_of_spec_fp8_peak": round(100.0 * value / world / SPEC_FP8_TFLOPS, 1)}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("bench.py: --gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    if world > 1:
+        os.environ.setdefault("NCCL_DEBUG", "INFO")
+        if torch.cuda.device_count() < world:
+            raise SystemExit("bench.py: %d ranks but %d visible GPUs" % (world, torch.cuda.device_count()))
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks, peak_kind = _peaks()
+
+    wl = make_workload(args.workload, args.m, seed_offset=rank)
+    set_bytes = input_set_bytes(wl)
+    res = measure(wl, dev, world, args.steps, args.warmup, args.accum, smi_id(local))
+    sm = summarize(wl, res, peaks, peak_kind, world)
+    step = res["step"]
+    A = res["accum"]
+    gemm_flops = sm["gemm_flops"]
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(wl, dev, K=min(K, 40), warmup=2, accum=A)
+        e2e = run_e2e(wl, dev, K=min(args.steps, e2e_steps(wl)), warmup=2, accum=A)
         if world > 1:
             t = torch.tensor([e2e["ms_per_step"]], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -337,98 +489,150 @@ def run_ours(args):
 
     bf16 = None
     if not args.no_bf16:
-        bms = bf16_step_ms(step, min(K, 200))
+        bms = bf16_step_ms(step, min(args.steps, 50))
         if world > 1:
             t = torch.tensor([bms], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             bms = float(t.item())
-        bf16 = {"ms_per_step": round(bms, 4),
-                "tflops": round(gemm_flops / (bms * 1e-3) / 1e12, 1),
-                "fp8_speedup": round(bms / ms_per_step, 3),
-                "what": "same step in BF16 via torch.matmul (cuBLAS), no quantization; "
-                        "fp8_speedup = BF16 step time / FP8 step time (quantizers included)"}
+        bf16 = bf16_summary(bms, res["ms_per_step"], gemm_flops)
+    del step, res["step"]
+    torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
+    del wl
+
+    sweep = None
+    if world == 1 and not args.no_sweep:
+        sweep = run_sweep(args, dev, peaks, peak_kind)
 
     if rank == 0:
         line = {
             "metric": METRIC,
-            "value": round(value, 2),
+            "value": round(sm["value"], 2),
             "unit": "TFLOP/s",
             "n_gpus": world,
-            "steps": K,
+            "steps": args.steps,
             "warmup": args.warmup,
-            "ms_per_step": round(ms_per_step, 4),
+            "ms_per_step": round(res["ms_per_step"], 4),
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": "e4m3",
             "data": "synthetic",
             "config": {
-                "workload": WORKLOAD,
-                "tokens_per_gpu": M_TOKENS, "hidden": 2048, "qkv_out": 3072, "o_out": 2048,
-                "seed": SEED,
-                "global_batch_tokens": M_TOKENS * world,
-                "l2": "3 rotating input sets of 132 MB each (> 126 MB L2)",
+                "workload": workload_tag(args.workload, args.m),
+                "layers": WORKLOADS[args.workload][2],
+                "tokens_per_gpu": args.m,
+                "seed": WORKLOADS[args.workload][1],
+                "global_batch_tokens": args.m * world,
+                "gemm_flops_per_step": gemm_flops,
+                "l2": "%d input set(s) of %.0f MB rotated: the inputs a step reads were last read "
+                      "at least 3 x 126 MB (L2) of inputs earlier" % (res["n_sets"], set_bytes / 1e6),
                 "parallelism": "dp%d (own batch per rank; FP32 dW all-reduce every %d steps)" % (world, A),
                 "step": "per layer: quant_act(X), fprop, quant_act(dY), and one launch for "
                         "dgrad + wgrad (dW added into FP32 main grads); quant_weight once per "
                         "%d-step accumulation window (the weights do not change within it)" % A,
-                "grad_exchange": "every %d steps: FP32 dW all-reduce across ranks (NCCL) and clear"
-                                 % A,
+                "grad_exchange": "every %d steps: FP32 dW all-reduce across ranks (NCCL) and clear" % A,
             },
-            "pct_fp8_peak": round(100.0 * value / world / fp8_peak_tf, 1),
-            "roofline": {
-                "bound": "tensor",
-                "kernel": "gemm_block_scaled_kernel (fprop/dgrad/wgrad, FLOP-weighted)",
-                "achieved": round(gemm_tf, 1),
-                "peak": round(fp8_peak_tf, 1),
-                "unit": "TFLOP/s",
-                "frac": round(gemm_tf / fp8_peak_tf, 4),
-                "peak_source": "%s: 2 x bf16_tflops_sustained (FP8 = 2 x BF16 nominal ratio)" % peak_kind,
-                "traffic": GEMM_TRAFFIC_BYTES,
-                "traffic_launch": "qkv.fprop (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-            },
-            "quantizers": {
-                "bound": "hbm", "achieved": round(quant_gbs, 1), "unit": "GB/s",
-                "peak": peaks["hbm_gbs"], "frac": round(quant_gbs / peaks["hbm_gbs"], 4),
-                "traffic": QUANT_TRAFFIC_BYTES,
-                "traffic_launch": "qkv.quant_x (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
-            },
-            "kernels": breakdown,
-            "gpu_launches": launches_timed,
-            "clocks": clocks,
-            "wall_ms_timed_region": round(total_ms, 3),
+            "pct_of_spec_fp8_peak": sm["pct_of_spec_fp8_peak"],
+            "roofline": sm["roofline"],
+            "quantizers": sm["quantizers"],
+            "time_split_ms_per_step": sm["time_split_ms_per_step"],
+            "kernels": sm["kernels"],
+            "gpu_launches": res["launches_timed"],
+            "clocks": res["clocks"],
+            "wall_ms_timed_region": round(res["total_ms"], 3),
             "timing": "K steps as CUDA graphs of %d steps plus the gradient exchange between them "
                       "(device events around it all); per-kernel times from a separate replay of %d "
-                      "steps with an event pair around every launch" % (A, K_inst),
+                      "steps with an event pair around every launch; clocks sampled over both"
+                      % (A, res["inst_steps"]),
         }
         if e2e is not None:
             line["e2e"] = {"value": e2e["value"], "unit": "TFLOP/s",
                            "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                           "ms_per_step": round(e2e["ms_per_step"], 3)}
+                           "ms_per_step": round(e2e["ms_per_step"], 3), "steps": e2e["steps"]}
         if cpu is not None:
             line["cpu_baseline"] = cpu
         if bf16 is not None:
             line["bf16_comparison"] = bf16
-            line["mfu_accounting"] = mfu_accounting(value / world, bf16["tflops"], peaks)
+            line["mfu_accounting"] = mfu_accounting(sm["value"] / world, bf16["tflops"], peaks)
         if ceiling is not None:
             if "tflops_step_shapes" in ceiling:
-                ceiling["gemm_vs_library_same_shapes"] = round(gemm_tf / ceiling["tflops_step_shapes"], 3)
+                ceiling["gemm_vs_library_same_shapes"] = round(sm["gemm_tf"] / ceiling["tflops_step_shapes"], 3)
             line["fp8_library_ceiling"] = ceiling
+        if sweep is not None:
+            line["sweep"] = sweep
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 
 
+def e2e_steps(wl) -> int:
+    """Steps of the end-to-end measure: about 40 at the attention-projection
+    size, fewer for larger workloads (their steps are PCIe-bound and long)."""
+    per = input_set_bytes(wl)
+    return max(6, min(40, int(40 * 2.7e8 / per)))
+
+
+def bf16_summary(bms, fp8_ms, gemm_flops):
+    return {"ms_per_step": round(bms, 4),
+            "tflops": round(gemm_flops / (bms * 1e-3) / 1e12, 1),
+            "fp8_speedup": round(bms / fp8_ms, 3),
+            "what": "same step in BF16 via torch.matmul (cuBLAS), no quantization; "
+                    "fp8_speedup = BF16 step time / FP8 step time (quantizers included)"}
+
+
+def run_sweep(args, dev, peaks, peak_kind):
+    """Short measurements of the other configurations (N = 1): the step rate,
+    the GEMM and quantizer rooflines, the FP8-vs-BF16 ratio, MFU accounting,
+    the end-to-end rate and the oracle baseline for each."""
+    import torch
+    out = {}
+    K = max(3, min(args.steps, 20))
+    for name, m in SWEEP:
+        if name == args.workload and m == args.m:
+            continue
+        wl = make_workload(name, m)
+        A = max(1, WINDOW_TOKENS // m)
+        res = measure(wl, dev, 1, K, max(3, min(args.warmup, 5)), A, smi_id(dev.index))
+        sm = summarize(wl, res, peaks, peak_kind, 1)
+        entry = {"ms_per_step": round(res["ms_per_step"], 4), "value": round(sm["value"], 1),
+                 "unit": "TFLOP/s", "steps": K, "accum": A,
+                 "gemm_tflops": round(sm["gemm_tf"], 1),
+                 "gemm_frac": sm["roofline"]["frac"],
+                 "gemm_frac_vs_spec": sm["roofline"]["frac_vs_spec"],
+                 "quant_gbs": sm["quantizers"]["achieved"],
+                 "quant_frac": sm["quantizers"]["frac"],
+                 "quant_act_frac": sm["quantizers"]["activations_only"]["frac"],
+                 "time_split_ms_per_step": sm["time_split_ms_per_step"],
+                 "kernels": sm["kernels"], "clocks": res["clocks"]}
+        if not args.no_bf16:
+            bms = bf16_step_ms(res["step"], K)
+            entry["bf16_comparison"] = bf16_summary(bms, res["ms_per_step"], sm["gemm_flops"])
+            entry["mfu_accounting"] = mfu_accounting(sm["value"], entry["bf16_comparison"]["tflops"], peaks)
+        del res["step"]
+        torch.cuda.empty_cache()
+        if not args.no_e2e:
+            e = run_e2e(wl, dev, K=min(K, e2e_steps(wl)), warmup=1, accum=A)
+            entry["e2e"] = {"value": round(sm["gemm_flops"] / (e["ms_per_step"] * 1e-3) / 1e12, 2),
+                            "unit": "TFLOP/s", "ms_per_step": round(e["ms_per_step"], 3),
+                            "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
+        torch.cuda.empty_cache()
+        if not args.no_cpu_baseline:
+            entry["cpu_baseline"] = cpu_baseline(wl, min_s=2.0)
+        out[workload_tag(name, m)] = entry
+        del wl
+    return out
+
+
 def bf16_step_ms(step, K):
     """The same linear step in BF16 through cuBLAS (torch.matmul): per layer
-    Y = X W^T, dX = dY W, dW = dY^T X, on the same rotating device input sets,
-    K steps captured in one CUDA graph and timed with device events.  This is
-    the FP8-vs-BF16 comparison of the pages' throughput claim, taken at the
-    level of the linear layer."""
+    Y = X W^T, dX = dY W, dW = dY^T X, on the same device input sets, K steps
+    captured in one CUDA graph and timed with device events.  This is the
+    FP8-vs-BF16 comparison of the pages' throughput claim, taken at the level
+    of the linear layers."""
     import torch
     outs = []
     for (x, w, dy) in step.sets[0]:
@@ -461,7 +665,7 @@ def bf16_step_ms(step, K):
     g.replay()
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / K
-    del g
+    del g, outs
     return ms
 
 
@@ -472,7 +676,7 @@ def mfu_accounting(fp8_tflops, bf16_tflops, peaks):
     projected throughput combines the measured FP8 linear-layer rate with the
     measured BF16 cuBLAS rate on the same shapes for the BF16 share."""
     f8, bf = 0.72, 0.28
-    nominal = {"fp8": 4500.0, "bf16": 2250.0}
+    nominal = {"fp8": SPEC_FP8_TFLOPS, "bf16": SPEC_BF16_TFLOPS}
     measured = {"fp8": 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "bf16": peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])}
     proj = 1.0 / (f8 / fp8_tflops + bf / bf16_tflops)
@@ -489,8 +693,8 @@ def mfu_accounting(fp8_tflops, bf16_tflops, peaks):
 def fp8_ceiling(wl, dev):
     """Library FP8 tensor-core throughput on this GPU, for context: cuBLASLt's
     MXFP8 GEMM (E4M3 operands, UE8M0 scales per 1x32 block, BF16 out) through
-    torch's scaled_mm, at 8192^3 and at the six GEMM shapes of the step.  Not
-    the same scaling granularity as the path (1x128 / 128x128), so it is a
+    torch's scaled_mm, at 8192^3 and at the GEMM shapes of the step.  Not the
+    same scaling granularity as the path (1x128 / 128x128), so it is a
     ceiling estimate, not a comparison arm.  None if unavailable."""
     import torch
     import torch.nn.functional as F
@@ -500,7 +704,7 @@ def fp8_ceiling(wl, dev):
     def rup(a, b):
         return (a + b - 1) // b * b
 
-    def timed(m, n, k, reps=20):
+    def timed(m, n, k, reps=10):
         # random operands: constant ones draw less power and run at clocks a
         # real GEMM does not keep (measured: 4.0 vs 2.6 PF/s at 8192^3)
         g = torch.Generator(device=dev).manual_seed(7)
@@ -526,6 +730,7 @@ def fp8_ceiling(wl, dev):
             s0.record(); f(); s1.record()
         torch.cuda.synchronize()
         ms = sorted(s0.elapsed_time(s1) for s0, s1 in ev)[reps // 2]
+        del a, b, sa, sb
         return ms
 
     try:
@@ -536,6 +741,7 @@ def fp8_ceiling(wl, dev):
             for (m, n, k) in ((L.m, L.n, L.k), (L.m, L.k, L.n), (L.n, L.k, L.m)):
                 tot_ms += timed(m, n, k)
                 tot_flops += 2 * m * n * k
+        torch.cuda.empty_cache()
         return {"source": "cuBLASLt MXFP8 via torch scaled_mm (1x32 UE8M0 scales, BF16 out)",
                 "tflops_8192cube": round(peak, 1),
                 "tflops_step_shapes": round(tot_flops / (tot_ms * 1e-3) / 1e12, 1)}
@@ -646,52 +852,78 @@ def run_e2e(wl, dev, K, warmup, accum):
     run(K)
     e.record()
     torch.cuda.synchronize()
+    if fp8.device_status() != 0:
+        raise RuntimeError("device status after the end-to-end run")
     windows = (K + accum - 1) // accum
-    return {"ms_per_step": s.elapsed_time(e) / K,
-            "h2d": int(bytes_in + bytes_w * windows / K),
-            "d2h": int(bytes_out + bytes_dw * windows / K)}
+    out = {"ms_per_step": s.elapsed_time(e) / K, "steps": K,
+           "h2d": int(bytes_in + bytes_w * windows / K),
+           "d2h": int(bytes_out + bytes_dw * windows / K)}
+    del host_w, host_in, host_out, host_dw, dev_w, dev_in, results, grads, wq
+    return out
 
 
 # ---------------------------------------------------------------- CPU oracle
 
-def _oracle_sample(wl, rows_per_gemm):
-    """The hot path on a bounded sample, through the CPU oracle: for every
-    layer, `rows_per_gemm` output rows of fprop, dgrad and wgrad, including the
-    quantization those rows need.  Returns the sampled GEMM FLOPs."""
+def oracle_threads() -> int:
+    """Gives the oracle's OpenMP loops every core this process may run on
+    (torchrun sets OMP_NUM_THREADS=1 for its ranks) and returns the number of
+    threads its parallel regions will use."""
+    import ctypes
+    import oracle
+    oracle._load()
+    n = len(os.sched_getaffinity(0))
+    try:
+        gomp = ctypes.CDLL("libgomp.so.1")
+    except OSError:
+        return 1 if os.environ.get("OMP_NUM_THREADS") == "1" else n
+    gomp.omp_set_num_threads(n)
+    return int(gomp.omp_get_max_threads())
+
+
+def _sample_idx(total, r):
     import numpy as np
+    return np.unique(np.linspace(0, total - 1, min(r, total)).astype(np.int64))
+
+
+def _oracle_sample(wl, r):
+    """The hot path on a bounded sample, through the CPU oracle: for every
+    layer, r output rows of fprop and of dgrad and an r x r block of wgrad's
+    output, each with the quantization those outputs need (the rows of X or dY
+    and the whole weight for fprop/dgrad; the r columns of dY and of X, over
+    all tokens, for wgrad).  Returns the sampled GEMM FLOPs."""
     import oracle
 
     flops = 0
     for L in wl.layers:
         m, n, k = L.m, L.n, L.k
-        r = rows_per_gemm
-        rows = np.linspace(0, m - 1, r).astype(np.int64)
+        rows = _sample_idx(m, r)
         oracle.linear_fprop(L.x[rows], L.w)
         oracle.linear_dgrad(L.dy[rows], L.w)
-        cols = np.linspace(0, n - 1, r).astype(np.int64)
-        oracle.linear_wgrad(L.dy[:, cols].contiguous(), L.x)
-        flops += 3 * 2 * r * n * k
+        ncols, kcols = _sample_idx(n, r), _sample_idx(k, r)
+        oracle.linear_wgrad(L.dy[:, ncols].contiguous(), L.x[:, kcols].contiguous())
+        flops += 2 * 2 * rows.size * n * k + 2 * ncols.size * kcols.size * m
     return flops
 
 
 def cpu_baseline(wl, min_s=10.0):
     """Times the oracle on a sample of the workload that takes at least `min_s`
-    seconds: the number of sampled output rows doubles until one sample run
-    lasts that long (the last run is the reported one, so it lasts between
-    `min_s` and about twice that)."""
-    n_cores = len(os.sched_getaffinity(0))
-    rows = 16
+    seconds: the sample size doubles until one sample run lasts that long (the
+    last run is the reported one, so it lasts between `min_s` and about twice
+    that)."""
+    n_cores = oracle_threads()
+    r = 16
     while True:
         t0 = time.perf_counter()
-        f = _oracle_sample(wl, rows)
+        f = _oracle_sample(wl, r)
         dt = time.perf_counter() - t0
-        if dt >= min_s or rows >= 8192:
+        if dt >= min_s or r >= 8192:
             break
-        rows *= 2
+        r *= 2
     return {"value": round(f / dt / 1e12, 6), "unit": "TFLOP/s", "cores": n_cores,
             "kind": "oracle",
-            "sample": "%d output rows of each of the 6 GEMMs (fprop/dgrad/wgrad x 2 layers) "
-                      "with the quantization they need, FP64 C oracle, %.1f s" % (rows, dt)}
+            "sample": "%d output rows of each fprop and dgrad and a %dx%d block of each wgrad "
+                      "(all layers) with the quantization they need, FP64 C oracle, %.1f s"
+                      % (r, r, r, dt)}
 
 
 def run_reference(args):
@@ -701,27 +933,27 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    from fp8_block_scaled_13_b200 import inputs
-    wl = inputs.attn_proj(seed=SEED, m=M_TOKENS)
-    rows = 8
+    wl = make_workload(args.workload, args.m)
+    n_cores = oracle_threads()
+    r = 8
     for _ in range(args.warmup):
-        _oracle_sample(wl, rows)
+        _oracle_sample(wl, r)
     t0 = time.perf_counter()
     flops = 0
     for _ in range(args.steps):
-        flops += _oracle_sample(wl, rows)
+        flops += _oracle_sample(wl, r)
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
-    n_cores = len(os.sched_getaffinity(0))
-    sample = ("%d output rows of each of the 6 GEMMs per step (fprop/dgrad/wgrad x 2 layers) "
-              "with the quantization they need, FP64 C oracle" % rows)
+    sample = ("%d output rows of each fprop and dgrad and a %dx%d block of each wgrad per step "
+              "(all layers) with the quantization they need, FP64 C oracle" % (r, r, r))
     line = {
         "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": WORKLOAD, "tokens_per_gpu": M_TOKENS, "hidden": 2048,
-                   "qkv_out": 3072, "o_out": 2048, "seed": SEED},
+        "config": {"workload": workload_tag(args.workload, args.m),
+                   "layers": WORKLOADS[args.workload][2], "tokens_per_gpu": args.m,
+                   "seed": WORKLOADS[args.workload][1]},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": n_cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -731,8 +963,43 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    args = _parse_args()
+# ---------------------------------------------------------------- launch
+
+def _free_port() -> int:
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def spawn_ranks(args, argv):
+    """--gpus N > 1 outside torchrun: start N ranks with torch.distributed.run
+    on this node, relay their output, and fail unless exactly one JSON line
+    for N GPUs came out."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node", str(args.gpus), "--master-addr", "127.0.0.1",
+           "--master-port", str(_free_port()), os.path.abspath(__file__)] + list(argv)
+    env = dict(os.environ)
+    if args.impl == "ours":
+        env.setdefault("NCCL_DEBUG", "INFO")
+    proc = subprocess.run(cmd, env=env, stdout=subprocess.PIPE, text=True, timeout=3600)
+    lines = [l for l in proc.stdout.splitlines() if l.startswith("{")]
+    for l in proc.stdout.splitlines():
+        print(l, flush=True)
+    if proc.returncode != 0:
+        return proc.returncode
+    if len(lines) != 1 or json.loads(lines[0]).get("n_gpus") != args.gpus:
+        print("bench.py: expected one JSON line for %d GPUs from the ranks" % args.gpus, file=sys.stderr)
+        return 1
+    return 0
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    args = _parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args, argv))
     if args.impl == "reference":
         run_reference(args)
     else:

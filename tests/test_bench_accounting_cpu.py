@@ -46,6 +46,51 @@ def test_quantizer_bytes_per_launch():
     assert costs["qkv.quant_weight"] == ("bytes", 3072 * 2048 * 4 + 24 * 16)
 
 
+def _full_block_shapes(m):
+    meta = dict(dtype=torch.bfloat16, device="meta")
+    layers = []
+    for name, n, k in (("qkv", 3072, 2048), ("o_proj", 2048, 2048), ("gate_up", 12288, 2048),
+                       ("down", 2048, 6144)):
+        layers.append(Linear(name, torch.empty(m, k, **meta), torch.empty(n, k, **meta),
+                             torch.empty(m, n, **meta)))
+    return Workload("full_block", 4, layers)
+
+
+def test_full_block_flops_per_step():
+    # fwd + bwd of the block: 3 GEMMs x 2*M*N*K per layer; at M = 32768,
+    # 6 * 32768 * (3072*2048 + 2048*2048 + 12288*2048 + 2048*6144) = 9.483 TFLOP
+    wl = _full_block_shapes(32768)
+    assert wl.gemm_flops() == 6 * 32768 * (3072 * 2048 + 2048 * 2048 + 12288 * 2048 + 2048 * 6144)
+    assert abs(wl.gemm_flops() / 1e12 - 9.4833) < 1e-3
+    # the per-M figures of the sweep: 1.185 / 2.315 / 4.742 TFLOP at M = 4096 / 8000 / 16384
+    for m, tf in ((4096, 1.1854), (8000, 2.3153), (16384, 4.7416)):
+        assert abs(_full_block_shapes(m).gemm_flops() / 1e12 - tf) < 1e-3
+    costs = bench._unit_costs(wl)
+    assert costs["gate_up.dgrad_wgrad"] == ("flops", 4 * 32768 * 12288 * 2048)
+    assert costs["down.quant_x"] == ("bytes", 32768 * 6144 * 4 + 2 * 32768 * 6144 // 128)
+
+
+def test_input_sets_cover_three_l2_capacities():
+    # 132 MB per attention-projection set: three sets; the 2.2 GB block: one
+    assert bench.n_input_sets(_attn_proj_shapes()) == 3
+    assert bench.n_input_sets(_full_block_shapes(32768)) == 1
+    assert bench.input_set_bytes(_full_block_shapes(32768)) == 2 * (
+        32768 * (2048 * 3 + 6144) + 32768 * (3072 + 2048 + 12288 + 2048)
+        + (3072 * 2048 + 2048 * 2048 + 12288 * 2048 + 2048 * 6144))
+
+
+def test_clock_summary_uses_loaded_samples():
+    idle = ["0", "1965", "1965", "120", "0", "Not Active", "Not Active", "Not Active", "Not Active"]
+    busy = ["0", "1800", "1965", "990", "100", "Not Active", "Not Active", "Not Active", "Active"]
+    busy2 = ["0", "1700", "1965", "1000", "98", "Not Active", "Not Active", "Not Active", "Active"]
+    out = bench.summarize_clocks([idle, busy, busy2, idle])
+    assert out["sm_mhz"] == 1750.0 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"] and out["samples_under_load"] == 2
+    # no loaded sample: fall back to all samples
+    out = bench.summarize_clocks([idle])
+    assert out["sm_mhz"] == 1965.0 and out["reasons"] == []
+
+
 def test_mfu_accounting_closed_forms():
     peaks = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6516.0}
     # at the measured peaks themselves the MFU against them is exactly 1

@@ -23,7 +23,8 @@ def test_reference_arm_json_line(oracle_mod):
     assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["steps"] == 1
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert d["config"]["workload"].startswith("attn_proj")
+    # the default workload: the full hidden-2048 / FFN-6144 block at 32768 tokens
+    assert d["config"]["workload"] == "full_block_m32768"
 
 
 def test_reference_arm_under_torchrun_prints_once(oracle_mod):
@@ -44,3 +45,28 @@ def test_reference_arm_under_torchrun_prints_once(oracle_mod):
     assert len(lines) == 1, out.stdout[-2000:]
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+
+
+def test_gpus_flag_without_torchrun_starts_the_ranks(oracle_mod):
+    """`bench.py --gpus 2` run directly (not under torchrun) starts two ranks
+    itself and prints one line for two GPUs."""
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--gpus", "2", "--steps", "1", "--warmup", "0", "--workload", "attn_proj",
+                          "--tokens", "1024"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["config"]["workload"] == "attn_proj_m1024"
+    # the oracle used every core of the host, not torchrun's one thread per rank
+    assert d["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))
+
+
+def test_gpus_flag_disagreeing_with_world_size_fails():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                          "--steps", "1"], capture_output=True, text=True, timeout=600, cwd=ROOT,
+                         env=env)
+    assert out.returncode != 0
+    assert "WORLD_SIZE" in (out.stderr + out.stdout)

@@ -1,12 +1,13 @@
 """Parity at the full workload sizes, in the launch configuration bench.py
-times: quantizers bit-exact on sampled rows / 128-row bands, GEMMs within
-tolerance on sampled output rows.
+times: quantizers bit-exact over the whole tensors, GEMMs within tolerance on
+sampled output rows.
 
 Workloads (fp8_block_scaled_13_b200/inputs.py): attention projections
 (M=8192, QKV 2048->3072, O 2048->2048), SwiGLU gate+up (M=16384,
 2048->12288, 8 channels x50), MLP down-projection with heavy tails
 (M=16384, 6144->2048, Student-t(3) activations, Laplace gradients, zero
-groups), and the full hidden-2048/FFN-6144 block at a ragged M=8000.
+groups), and the full hidden-2048/FFN-6144 block at M = 4096, 8000 (ragged),
+16384 and 32768 tokens.
 """
 import numpy as np
 import pytest
@@ -29,8 +30,8 @@ def fp8():
 
 def _workload(name):
     from fp8_block_scaled_13_b200 import inputs
-    if name == "full_block_m8000":
-        return inputs.full_block(seed=4, m=8000)
+    if name.startswith("full_block_m"):
+        return inputs.full_block(seed=4, m=int(name[len("full_block_m"):]))
     return inputs.WORKLOADS[name]()
 
 
@@ -52,25 +53,34 @@ def _check_layer(fp8, oracle_mod, L, seed):
     assert fp8.device_status() == 0
     m, n, k = L.m, L.n, L.k
 
-    # ---- quantizers: weight in full, activations on sampled rows / bands
+    # ---- quantizers, whole tensors: the weight (codes, compact scales,
+    # transpose, both expanded scale copies) and both activations in both
+    # layouts (codes, scale bytes, zero padding of the transposed rows)
     oq, os_ = oracle_mod.quant_weight(L.w)
     assert np.array_equal(np_u8(wq.s), os_) and np.array_equal(np_u8(wq.q), oq)
     assert np.array_equal(np_u8(wq.qt), oq.T)
     assert np.array_equal(unblock(wq.s_fwd, n, k // 128), np.repeat(os_, 128, axis=0))
     assert np.array_equal(unblock(wq.s_bwd, k, n // 128), np.repeat(os_.T, 128, axis=0))
-    rows = _sample(m, 64, seed)
-    for src, q in ((L.x, xq), (L.dy, dyq)):
+    del oq, os_
+    nb = (m + 127) // 128
+    for what, src, q in (("X", L.x, xq), ("dY", L.dy, dyq)):
         cols = src.shape[1]
-        oq, os_ = oracle_mod.quant_rowwise(src[rows])
-        assert np.array_equal(np_u8(q.q)[rows], oq)
-        assert np.array_equal(unblock(q.s, m, cols // 128)[rows], os_)
-        nb = (m + 127) // 128
-        st_all = unblock(q.st, cols, nb)
-        for b in sorted({0, nb - 1, int(seed) % nb}):
-            r0, r1 = b * 128, min(m, b * 128 + 128)
-            oqt, ost = oracle_mod.quant_colwise(src[r0:r1])
-            assert np.array_equal(np_u8(q.qt)[:, r0:r1], oqt)
-            assert np.array_equal(st_all[:, b], ost[:, 0])
+        oq, os_ = oracle_mod.quant_rowwise(src)
+        assert np.array_equal(unblock(q.s, m, cols // 128), os_), "%s %s row scales" % (L.name, what)
+        assert np.array_equal(np_u8(q.q), oq), "%s %s row codes" % (L.name, what)
+        del oq, os_
+        oqt, ost = oracle_mod.quant_colwise(src)
+        qt_full = np_u8(q.qt)
+        st = unblock(q.st, cols, nb)
+        assert np.array_equal(st, ost), "%s %s column scales" % (L.name, what)
+        assert np.array_equal(qt_full[:, :m], oqt), "%s %s column codes" % (L.name, what)
+        assert not qt_full[:, m:(m + 15) // 16 * 16].any(), "%s %s padding" % (L.name, what)
+        # every all-zero 128-token band: the zero-amax scale byte and zero codes
+        zero_bands = [b for b in range(nb) if not src[b * 128:(b + 1) * 128].view(torch.int16).any()]
+        for b in zero_bands:
+            assert (st[:, b] == 127).all()
+            assert (qt_full[:, b * 128:min(m, b * 128 + 128)] == 0).all()
+        del oqt, ost, qt_full, st
 
     # ---- GEMMs on sampled output rows
     rows = _sample(m, N_ROWS, seed + 1)
@@ -106,9 +116,20 @@ def test_single_fprop_full(fp8, oracle_mod, name):
 
 
 @pytest.mark.parametrize("name", ["attn_proj", "swiglu_gate_up", "mlp_down_heavy",
-                                  "full_block_m8000"])
-def test_workload_sampled(fp8, oracle_mod, name):
+                                  "full_block_m4096", "full_block_m8000", "full_block_m16384",
+                                  "full_block_m32768"])
+def test_workload(fp8, oracle_mod, name):
     wl = _workload(name)
     for i, L in enumerate(wl.layers):
         _check_layer(fp8, oracle_mod, L, seed=17 * i + len(name))
         torch.cuda.empty_cache()
+
+
+def test_mlp_down_heavy_has_zero_bands():
+    """The heavy-tailed workload holds the zero 128-token bands that the
+    column-wise zero-amax checks above run over, in X and in dY."""
+    L = _workload("mlp_down_heavy").layers[0]
+    for src in (L.x, L.dy):
+        nb = src.shape[0] // 128
+        zero = [b for b in range(nb) if not src[b * 128:(b + 1) * 128].view(torch.int16).any()]
+        assert len(zero) == 8

@@ -78,11 +78,37 @@ def test_quant_act_adversarial_groups(fp8, oracle_mod):
     x[20, 384:512] = 1.0
     x[20, 400] = 3.0e38                                # near BF16 max
     x[21, 512:640] = torch.arange(128) * 2.0 ** -133   # smallest subnormals
-    x[22:150, 640:768] = 0.0                           # a zero 128-row band (colwise zero group)
+    x[22:150, 640:768] = 0.0                           # zero rows straddling two 128-row groups
+    x[128:256, 1152:1280] = 0.0                        # an aligned zero 128-row group in 128 columns
+    x[128:256, 1100] = -0.0                            # a column group of negative zeros
     x[30, 768:896] = 224.0                             # half of 448: exponent boundary
     x[31, 768:896] = 1.75                              # 1.75 = 448 * 2^-8
     x[32, 768:896] = 1.78125
-    _check_all(fp8, oracle_mod, x.to(torch.bfloat16), "both")
+    xq = _check_all(fp8, oracle_mod, x.to(torch.bfloat16), "both")
+    # the zero-amax path of the column-wise quantizer, byte by byte: scale
+    # byte 127 (e = 0) and codes 0x00 (or 0x80 for -0) in the zero groups
+    qt, st, _ = gpu_colwise(xq)
+    assert (st[1152:1280, 1] == 127).all()
+    assert (qt[1152:1280, 128:256] == 0).all()
+    assert st[1100, 1] == 127 and (qt[1100, 128:256] == 0x80).all()
+    # and the row-wise zero groups
+    q, s = gpu_rowwise(xq)
+    assert s[0, 0] == 127 and (q[0, 0:128] == 0).all()
+    assert s[1, 0] == 127 and (q[1, 0:128] == 0x80).all()
+
+
+def test_quant_act_zero_ragged_column_group(fp8, oracle_mod):
+    """A short last token group (300 rows: 44 in the third group) that is all
+    zero in some columns, and an aligned full zero group, in every layout."""
+    x = _rand((300, 384), 21).float()
+    x[256:300, 0:64] = 0.0         # the short last group of columns 0..63
+    x[128:256, 128:256] = 0.0      # a full 128-row group of columns 128..255
+    for layout in ("colwise", "both"):
+        xq = _check_all(fp8, oracle_mod, x.to(torch.bfloat16), layout)
+        qt, st, pad = gpu_colwise(xq)
+        assert (st[0:64, 2] == 127).all() and (qt[0:64, 256:300] == 0).all()
+        assert (st[128:256, 1] == 127).all() and (qt[128:256, 128:256] == 0).all()
+        assert (st[64:, 2] != 127).any()   # the other columns' last groups are not zero
 
 
 def test_quant_act_strided_input(fp8, oracle_mod):

@@ -37,8 +37,8 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool checked = false;
   bool supported = false;
+  int index = 0;  // CUDA device ordinal (index into the per-device caches)
   int sms = 0;
-  bool attrs_set = false;
 };
 
 std::mutex g_mu;
@@ -65,6 +65,7 @@ int current_device(DeviceInfo** out) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return PURO_ERR_CUDA;
     d.supported = (major == 10 && minor == 0);
+    d.index = dev;
     d.sms = sms;
     d.checked = true;
   }
@@ -125,8 +126,8 @@ int launch_status() {
 // ------------------------------------------------------------------ quant
 
 template <bool ROW, bool COL, bool BLOCK, bool RSHFL>
-int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, int sms,
-                 cudaStream_t stream) {
+int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, const DeviceInfo& dev,
+                     cudaStream_t stream) {
   int st = get_encoder();
   if (st != PURO_OK) return st;
   // BF16 input as a 2-D tensor of 16-bit elements {cols, rows}, 128 x 128 boxes
@@ -143,14 +144,12 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, in
   constexpr uint32_t smem = puro::quant_smem_bytes();
   // per device, once (threads racing on the first call both set the same value)
   static std::atomic<bool> attr_done[kMaxDevices] = {};
-  int dev_id = 0;
-  cudaGetDevice(&dev_id);
-  if (!attr_done[dev_id].load(std::memory_order_acquire)) {
+  if (!attr_done[dev.index].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return PURO_ERR_CUDA;
-    attr_done[dev_id].store(true, std::memory_order_release);
+    attr_done[dev.index].store(true, std::memory_order_release);
   }
-  const int64_t grid = p.tiles < 2 * (int64_t)sms ? p.tiles : 2 * (int64_t)sms;
+  const int64_t grid = p.tiles < 2 * (int64_t)dev.sms ? p.tiles : 2 * (int64_t)dev.sms;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -168,11 +167,11 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, in
 // Row scales by shuffles when each CTA has few tiles (measured faster up to
 // about 8 tiles per CTA; the redundant per-thread form wins on long streams).
 template <bool ROW, bool COL, bool BLOCK>
-int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, int sms,
+int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, const DeviceInfo& dev,
                  cudaStream_t stream) {
-  if (ROW && !BLOCK && p.tiles <= 8 * 2 * (int64_t)sms)
-    return launch_quant_cfg<ROW, COL, BLOCK, true>(x, ld_x, p, sms, stream);
-  return launch_quant_cfg<ROW, COL, BLOCK, false>(x, ld_x, p, sms, stream);
+  if (ROW && !BLOCK && p.tiles <= 8 * 2 * (int64_t)dev.sms)
+    return launch_quant_cfg<ROW, COL, BLOCK, true>(x, ld_x, p, dev, stream);
+  return launch_quant_cfg<ROW, COL, BLOCK, false>(x, ld_x, p, dev, stream);
 }
 
 // ------------------------------------------------------------------ gemm
@@ -260,8 +259,7 @@ int launch_gemm_cfg(const GemmArgs& g0, const GemmArgs* g1, DeviceInfo* dev, cud
   auto kern = puro::gemm_block_scaled_kernel<CG, BN, BK, OUT0, OUT1>;
   // per device, once (threads racing on the first call both store the same value)
   static std::atomic<int> max_clusters[kMaxDevices] = {};
-  int dev_id = 0;
-  cudaGetDevice(&dev_id);
+  const int dev_id = dev->index;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -495,9 +493,9 @@ int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, 
   p.tiles_c = (int32_t)(cols / 128);
   p.tiles = (int32_t)(p.tiles_c * ((rows + 127) / 128));
   cudaStream_t sm = static_cast<cudaStream_t>(stream);
-  if (row && col) return launch_quant<true, true, false>(x, ld_x, p, dev->sms, sm);
-  if (row) return launch_quant<true, false, false>(x, ld_x, p, dev->sms, sm);
-  return launch_quant<false, true, false>(x, ld_x, p, dev->sms, sm);
+  if (row && col) return launch_quant<true, true, false>(x, ld_x, p, *dev, sm);
+  if (row) return launch_quant<true, false, false>(x, ld_x, p, *dev, sm);
+  return launch_quant<false, true, false>(x, ld_x, p, *dev, sm);
 }
 
 int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, void* q, int64_t ld_q,
@@ -529,8 +527,8 @@ int puro_fp8_quant_weight(const void* w, int64_t n, int64_t k, int64_t ld_w, voi
   p.tiles_c = (int32_t)(k / 128);
   p.tiles = (int32_t)(p.tiles_c * (n / 128));
   cudaStream_t sm = static_cast<cudaStream_t>(stream);
-  if (qt) return launch_quant<true, true, true>(w, ld_w, p, dev->sms, sm);
-  return launch_quant<true, false, true>(w, ld_w, p, dev->sms, sm);
+  if (qt) return launch_quant<true, true, true>(w, ld_w, p, *dev, sm);
+  return launch_quant<true, false, true>(w, ld_w, p, *dev, sm);
 }
 
 int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx, const void* qw,

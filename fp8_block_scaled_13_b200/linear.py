@@ -104,6 +104,40 @@ def _require(t: torch.Tensor, dtype, name: str):
         raise ValueError("%s must be a row-major 2-D tensor" % name)
 
 
+def _check_row_operand(qa: "QuantAct", name: str):
+    """The row-wise codes [rows, cols] and blocked scales (rows x cols/128
+    groups) of a QuantAct, sized for the kernel's tensor maps."""
+    q = _need(qa.q, "%s was quantized without the row-wise layout" % name)
+    _check_tensor(q, (qa.rows, qa.cols), (torch.uint8,), name + ".q", min_cols=True)
+    _check_bytes(_need(qa.s, "%s has no row-wise scales" % name),
+                 blocked_scale_bytes(qa.rows, qa.cols // 128), name + ".s")
+
+
+def _check_col_operand(qa: "QuantAct", name: str):
+    """The transposed codes [cols, >= rows rounded to 16] and blocked scales
+    (cols x ceil(rows/128) groups) of a QuantAct."""
+    qt = _need(qa.qt, "%s was quantized without the column-wise layout" % name)
+    _check_tensor(qt, (qa.cols, _round16(qa.rows)), (torch.uint8,), name + ".qt", min_cols=True)
+    _check_bytes(_need(qa.st, "%s has no column-wise scales" % name),
+                 blocked_scale_bytes(qa.cols, (qa.rows + 127) // 128), name + ".st")
+
+
+def _check_weight(wq: "QuantWeight", fwd: bool):
+    """The weight codes and the blocked scales of the GEMM that reads them:
+    q [n, k] with s_fwd (n x k/128 groups) for fprop, qt [k, n] with s_bwd
+    (k x n/128 groups) for dgrad."""
+    if fwd:
+        _check_tensor(wq.q, (wq.n, wq.k), (torch.uint8,), "wq.q", min_cols=True)
+        _check_bytes(_need(wq.s_fwd, "the weight was quantized without its blocked fprop scales"),
+                     blocked_scale_bytes(wq.n, wq.k // 128), "wq.s_fwd")
+    else:
+        if wq.qt is None or wq.s_bwd is None:
+            raise ValueError("the weight was quantized without its transposed copy "
+                             "(quant_weight(transpose=True))")
+        _check_tensor(wq.qt, (wq.k, wq.n), (torch.uint8,), "wq.qt", min_cols=True)
+        _check_bytes(wq.s_bwd, blocked_scale_bytes(wq.k, wq.n // 128), "wq.s_bwd")
+
+
 @dataclass
 class QuantAct:
     """Result of quant_act.  rows/cols describe the BF16 input."""
@@ -203,8 +237,8 @@ def gemm_fprop(xq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) -
     m, k, n = xq.rows, xq.cols, wq.n
     if wq.k != k:
         raise ValueError("inner dimensions differ: %d vs %d" % (k, wq.k))
-    _need(xq.q, "X was quantized without the row-wise layout fprop needs")
-    _need(wq.s_fwd, "the weight was quantized without its blocked fprop scales")
+    _check_row_operand(xq, "xq")
+    _check_weight(wq, fwd=True)
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=xq.q.device)
     _check_tensor(out, (m, n), (torch.bfloat16,), "out", min_cols=False)
@@ -222,9 +256,8 @@ def gemm_dgrad(dyq: QuantAct, wq: QuantWeight, out: torch.Tensor | None = None) 
     m, n, k = dyq.rows, dyq.cols, wq.k
     if wq.n != n:
         raise ValueError("dY has %d columns, W has %d rows" % (n, wq.n))
-    if wq.qt is None or wq.s_bwd is None:
-        raise ValueError("dgrad needs the transposed weight codes (quant_weight(transpose=True))")
-    _need(dyq.q, "dY was quantized without the row-wise layout dgrad needs")
+    _check_weight(wq, fwd=False)
+    _check_row_operand(dyq, "dyq")
     if out is None:
         out = torch.empty((m, k), dtype=torch.bfloat16, device=dyq.q.device)
     _check_tensor(out, (m, k), (torch.bfloat16,), "out")
@@ -247,11 +280,11 @@ def gemm_wgrad(dyq: QuantAct, xq: QuantAct, out: torch.Tensor | None = None,
     m, n, k = dyq.rows, dyq.cols, xq.cols
     if xq.rows != m:
         raise ValueError("dY and X have different token counts")
-    _need(dyq.qt, "dY was quantized without the column-wise layout wgrad needs")
-    _need(xq.qt, "X was quantized without the column-wise layout wgrad needs")
+    if out is None and accumulate:
+        raise ValueError("accumulate=True needs the FP32 buffer to add into")
+    _check_col_operand(dyq, "dyq")
+    _check_col_operand(xq, "xq")
     if out is None:
-        if accumulate:
-            raise ValueError("accumulate=True needs the FP32 buffer to add into")
         out = torch.empty((n, k), dtype=torch.bfloat16, device=dyq.qt.device)
     _check_tensor(out, (n, k), (torch.bfloat16, torch.float32), "out")
     if out.dtype == torch.float32:
@@ -280,11 +313,12 @@ def gemm_dgrad_wgrad(dyq: QuantAct, wq: QuantWeight, xq: QuantAct, dx: torch.Ten
     m, n, k = dyq.rows, dyq.cols, wq.k
     if wq.n != n or xq.rows != m or xq.cols != k:
         raise ValueError("shapes of dY, W and X do not agree")
-    if wq.qt is None or wq.s_bwd is None:
-        raise ValueError("the weight was quantized without its transposed copy")
-    _need(dyq.q, "dY was quantized without the row-wise layout dgrad needs")
-    _need(dyq.qt, "dY was quantized without the column-wise layout wgrad needs")
-    _need(xq.qt, "X was quantized without the column-wise layout wgrad needs")
+    if dw is None and accumulate:
+        raise ValueError("accumulate=True needs the FP32 buffer to add into")
+    _check_weight(wq, fwd=False)
+    _check_row_operand(dyq, "dyq")
+    _check_col_operand(dyq, "dyq")
+    _check_col_operand(xq, "xq")
     dev = dyq.q.device
     if dx is None:
         dx = torch.empty((m, k), dtype=torch.bfloat16, device=dev)

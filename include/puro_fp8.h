@@ -85,14 +85,15 @@ enum {
 };
 
 /* Bytes of a blocked scale array for `rows` rows and `groups` groups
- * (ceil(rows/128) * ceil(groups/4) * 512); 0 if either is <= 0. */
+ * (ceil(rows/128) * ceil(groups/4) * 512); 0 if either is <= 0.  A support
+ * call of this library's storage layout; the pages have no counterpart. */
 PURO_API int64_t puro_fp8_blocked_scale_bytes(int64_t rows, int64_t groups);
 
 /*
  * puro_fp8_quant_act -- online 1x128 quantization of an activation or
- * gradient (the "activations and gradients, one scale per 128 elements along
- * the reduction direction" rule of ta-paperlens §3.2 and the 1-D groups of
- * paper.rainbus.top step (3)).
+ * gradient: one scale for every 128 consecutive values along the GEMM
+ * reduction dimension, for activations and for gradients alike (ta-paperlens
+ * explainer §3.2; the 1-D groups of paper.rainbus.top, "方法步骤详情" step (3)).
  *
  * x      : BF16 [rows, cols], row stride ld_x elements (ld_x >= cols).
  * layout : PURO_ROWWISE, PURO_COLWISE or PURO_BOTH.  cols % 128 == 0.
@@ -116,9 +117,10 @@ PURO_API int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64
                                 void* qt, int64_t ld_qt, void* st, void* stream);
 
 /*
- * puro_fp8_quant_weight -- 128x128 block quantization of a weight
- * (paper.rainbus.top background and step (3): "weights in 128x128 blocks,
- * one online power-of-two scale each").
+ * puro_fp8_quant_weight -- 128x128 block quantization of a weight: one
+ * power-of-two scale, computed online, for each 128x128 block
+ * (paper.rainbus.top summary, background "FP8 块级混合精度训练" and
+ * "方法步骤详情" step (3)).
  *
  * w     : BF16 [n, k], row stride ld_w elements; n % 128 == 0, k % 128 == 0.
  * q     : E4M3 [n, k], row stride ld_q bytes.
@@ -152,7 +154,12 @@ PURO_API int puro_fp8_gemm_fprop(const void* qx, int64_t ld_qx, const void* sx,
                                  void* stream);
 
 /*
- * puro_fp8_gemm_dgrad -- dX = dY W (data-gradient GEMM, reduction over n).
+ * puro_fp8_gemm_dgrad -- dX = dY W, the data-gradient GEMM (paperlayer.ai
+ * summary, Appendix C "FP8 implementation pipeline": the forward,
+ * data-gradient and weight-gradient GEMMs all run in blockwise E4M3;
+ * paper.rainbus.top summary, "方法步骤详情" step (3): Dgrad in E4M3).  Its
+ * reduction runs over n, so dY carries its 1x128 row-wise groups along n and
+ * the weight its 128x128 blocks, read through the transposed codes.
  * qdy : E4M3 [m, n] (ld_qdy), sdy   : blocked, m rows x n/128 groups (quant_act ROWWISE of dY)
  * qwt : E4M3 [k, n] (ld_qwt), sw_bwd: blocked, k rows x n/128 groups (quant_weight qt, s_bwd)
  * dx  : BF16 [m, k], row stride ld_dx elements.
@@ -207,8 +214,9 @@ enum {
 };
 
 /*
- * puro_fp8_gemm_dgrad_wgrad -- the two backward GEMMs of one linear layer in
- * one launch: dX = dY W (arguments and result exactly as puro_fp8_gemm_dgrad)
+ * puro_fp8_gemm_dgrad_wgrad -- the two backward GEMMs of one linear layer
+ * (the data- and weight-gradient GEMMs of paperlayer.ai Appendix C) in one
+ * launch: dX = dY W (arguments and result exactly as puro_fp8_gemm_dgrad)
  * and dW = dY^T X (as puro_fp8_gemm_wgrad, or the FP32 forms, by dw_kind).
  * The two are independent given the quantized dY, X and W.  Sharing the launch
  * only changes which SM computes which output tile: the tiles of both are
@@ -230,6 +238,9 @@ PURO_API int puro_fp8_gemm_dgrad_wgrad(const void* qdy, int64_t ld_qdy, const vo
                                        void* stream);
 
 /*
+ * Support calls (error reporting and self-tests of this library; the pages
+ * have no counterpart).
+ *
  * puro_fp8_device_status -- synchronizes `stream`, then returns and clears the
  * library's device error word for the current device: PURO_OK, or
  * PURO_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the last

@@ -220,3 +220,30 @@ def test_wrapper_rejects_missing_layouts_and_bad_buffers(fp8):
     # group slot are left as they were
     assert np.array_equal(gpu_rowwise(again)[1], gpu_rowwise(x_row)[1])
     assert fp8.device_status() == 0
+
+
+def test_wrapper_rejects_short_scale_buffers(fp8):
+    """A QuantAct or QuantWeight whose scale buffers are smaller than their
+    blocked layout (a caller-built or reused result) is refused before the
+    launch: the kernel's tensor maps would read past the buffers' ends."""
+    import dataclasses
+    x, w, dy = _layer(256, 256, 384, 22)
+    dev = torch.device("cuda")
+    x, w, dy = x.to(dev), w.to(dev), dy.to(dev)
+    xq = fp8.quant_act(x, "both")
+    dyq = fp8.quant_act(dy, "both")
+    wq = fp8.quant_weight(w)
+    short = lambda t: t[: t.numel() - 16]
+    with pytest.raises(ValueError, match="bytes"):
+        fp8.gemm_fprop(dataclasses.replace(xq, s=short(xq.s)), wq)
+    with pytest.raises(ValueError, match="bytes"):
+        fp8.gemm_fprop(xq, dataclasses.replace(wq, s_fwd=short(wq.s_fwd)))
+    with pytest.raises(ValueError, match="bytes"):
+        fp8.gemm_dgrad(dyq, dataclasses.replace(wq, s_bwd=short(wq.s_bwd)))
+    with pytest.raises(ValueError, match="bytes"):
+        fp8.gemm_wgrad(dataclasses.replace(dyq, st=short(dyq.st)), xq)
+    with pytest.raises(ValueError, match="bytes"):
+        fp8.gemm_dgrad_wgrad(dyq, wq, dataclasses.replace(xq, st=short(xq.st)))
+    with pytest.raises(ValueError):
+        fp8.gemm_fprop(dataclasses.replace(xq, q=xq.q[:, :256]), wq)    # codes narrower than K
+    assert fp8.device_status() == 0

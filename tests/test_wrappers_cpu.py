@@ -49,3 +49,4 @@ def test_shape_and_layout_errors():
         fp8.gemm_wgrad(fp8.QuantAct(128, 128, qt=torch.zeros(128, 128, dtype=torch.uint8)),
                        fp8.QuantAct(128, 128, qt=torch.zeros(128, 128, dtype=torch.uint8)),
                        accumulate=True)
+

@@ -20,35 +20,37 @@
 //   COL   : column amax by a shuffle + shared-memory reduction over the 8
 //           warps; codes transposed through an XOR-swizzled 16 KB shared tile
 //           (conflict-free 8-byte writes, 16-byte reads) and written out as
-//           128-byte rows of the transposed matrix.
+//           128-byte rows of the transposed matrix.  The transposed tile is
+//           double-buffered and copied out during the next tile, after the
+//           barrier every tile starts with anyway.
 //   BLOCK : one amax over the whole tile (128x128 weight block); codes written
 //           in place and, optionally, transposed.
-// The amax is taken on the integer BF16 magnitude bits (|x| is itself a BF16,
+// Per tile the block meets at three barriers: stage consumed (which also
+// publishes the previous tile's transposed codes), column partial maxima
+// published, column scales published.  The column scales are reduced by 64
+// threads while the others already encode their rows.
+// The amax is taken with the max-of-absolute-values instruction on BF16
+// pairs and then compared as integer magnitude bits (|x| is itself a BF16,
 // and the order of non-negative floats equals the order of their bits), and
-// the scale exponent comes from the exponent/mantissa fields alone: with
-// amax = 1.f * 2^E, e = E - 8 if 1.f <= 1.75 (mantissa bits <= 0x60), else
-// E - 7.  Scaling by 2^-e is an exact packed FP32 multiply (no flush to zero:
-// this file must not be built with fast-math), followed by one hardware
-// round-to-nearest-even, saturating conversion to E4M3 per value.
+// the scale exponent comes from the exponent/mantissa fields alone, two
+// groups per 32-bit word: with amax = 1.f * 2^E, e = E - 8 if 1.f <= 1.75
+// (mantissa bits <= 0x60), else E - 7.  Scaling by 2^-e is an exact packed
+// FP32 multiply (no flush to zero: this file must not be built with
+// fast-math), followed by one hardware round-to-nearest-even, saturating
+// conversion to E4M3 per value.
 #pragma once
 
 #include "common.cuh"
 
 namespace puro {
 
-#ifndef PURO_QUANT_RPT
-#define PURO_QUANT_RPT 8
-#endif
-// rows of the 128x128 tile per thread (each thread holds RPT rows x 8 columns;
-// 16 threads cover a row, 128/RPT row groups cover the tile).  8 (256 threads,
-// two CTAs per SM) was measured faster than 4 (512 threads, 64 registers) for
-// the BOTH layout at every size tried (8192x3072: 20.9 vs 22.8 us; 16384x12288:
-// 147 vs 162 us) and equal within a few % for the single layouts.
-constexpr int kQRpt = PURO_QUANT_RPT;
-static_assert(kQRpt == 4 || kQRpt == 8, "4 or 8 rows per thread");
-constexpr int kQThreads = 16 * 128 / kQRpt;
+// 256 threads: 16 threads cover a 128-column row chunk (8 columns each) and
+// 16 row groups of 8 rows cover the 128-row tile.  (4 rows per thread with 512
+// threads and 64 registers was measured slower for the BOTH layout.)
+constexpr int kQThreads = 256;
 constexpr int kQStages = 2;
 constexpr uint32_t kQTileBytes = 128 * 128 * 2;
+constexpr uint32_t kQtTileBytes = 128 * 128;  // one transposed code tile
 
 struct QuantParams {
   int64_t rows, cols;
@@ -68,21 +70,30 @@ struct QuantParams {
   int32_t tiles_c, tiles;
 };
 
-// Scale exponent from the BF16 bits of a group's amax (sign already cleared).
-__device__ __forceinline__ int scale_exponent_from_bits(uint32_t a) {
-  if (a == 0) return 0;
-  const int ef = static_cast<int>(a >> 7);  // biased exponent field
-  if (ef == 0) return -127;                 // subnormal amax: always clamps
-  const int e = ef - 127 - 8 + ((a & 0x7Fu) > 0x60u ? 1 : 0);
-  return e < -127 ? -127 : e;
+// Scale exponents of two groups at once.  a2 holds two amax magnitudes (BF16
+// bits, sign cleared) in its 16-bit halves; each half of the result is
+// k = 127 - e, the FP32 exponent field of 2^-e: with t the biased exponent
+// field and c = (mantissa > 0x60), e = t - 135 + c, clamped to e >= -127
+// (k <= 254; a subnormal amax always clamps).  The largest finite BF16 gives
+// k = 7, so no upper clamp is needed.  A zero amax also comes out as
+// k = 254; its codes are zero for any scale, and its scale byte is fixed up
+// by scale_bytes2.
+__device__ __forceinline__ uint32_t scale_k2(uint32_t a2) {
+  const uint32_t t2 = (a2 >> 7) & 0x00FF00FFu;
+  const uint32_t c2 = (((a2 & 0x007F007Fu) + 0x001F001Fu) >> 7) & 0x00010001u;
+  return __vminu2(0x01060106u - t2 - c2, 0x00FE00FEu);
 }
 
-// 2^-e as an FP32 (e in [-127, 120], so the result is a normal number), in
-// both lanes of a float2.
-__device__ __forceinline__ float2 pow2_neg_x2(int e) {
-  const float f = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
-  return make_float2(f, f);
+// UE8M0 scale bytes e + 127 = 254 - k of the two groups of scale_k2, with the
+// zero-amax rule (e = 0, byte 127) applied; one byte in each 16-bit half.
+__device__ __forceinline__ uint32_t scale_bytes2(uint32_t a2, uint32_t k2) {
+  const uint32_t z2 = __vcmpeq2(a2, 0u);
+  return ((0x00FE00FEu - k2) & ~z2) | (0x007F007Fu & z2);
 }
+
+// 2^-e of the low / high group of scale_k2 as an FP32.
+__device__ __forceinline__ float scale_lo(uint32_t k2) { return __uint_as_float(k2 << 23); }
+__device__ __forceinline__ float scale_hi(uint32_t k2) { return __uint_as_float((k2 << 7) & 0x7F800000u); }
 
 // Four values (pairs a, b) times 2^-e (s2) -> four E4M3 codes in one word,
 // a.x in the low byte.  The packed multiply is exact (a power of two,
@@ -124,12 +135,6 @@ __device__ __forceinline__ uint2 encode_row8(const uint4& v, float2 s2) {
   return o;
 }
 
-// Four codes of column l of rows 0..3 of the thread's block, scaled by s2.
-__device__ __forceinline__ uint32_t encode_col4(const uint4 (&v)[4], int l, float2 s2) {
-  return encode4(make_float2(elem_f32(v[0], l), elem_f32(v[1], l)),
-                 make_float2(elem_f32(v[2], l), elem_f32(v[3], l)), s2);
-}
-
 // Eight codes of column l of the thread's 8x8 block (rows 0..7), scaled by s2.
 __device__ __forceinline__ uint2 encode_col8(const uint4 (&v)[8], int l, float2 s2) {
   uint2 o;
@@ -140,21 +145,17 @@ __device__ __forceinline__ uint2 encode_col8(const uint4 (&v)[8], int l, float2 
   return o;
 }
 
-// Column l of the thread's block as codes into its transposed-tile row `row`.
-// 8 rows per thread: 8 codes at 8-byte chunk i ^ 2(j & 7), so that a 16-byte
-// unit holds two consecutive chunks in order (one plain 16-byte load per 16
-// rows on the way out) while the 32 stores of a warp still fill 16 distinct
-// chunk positions twice (two wavefronts, the minimum for 256 bytes).
-// 4 rows per thread: 4 codes at 4-byte slot i ^ 2j (conflict-free; the
-// readout swaps the 8-byte halves of odd column groups).
-__device__ __forceinline__ void put_col_codes(uint8_t* row, const uint4 (&v)[8], int l, float2 s2,
-                                              int i, int j) {
-  *reinterpret_cast<uint2*>(row + ((i ^ (2 * (j & 7))) << 3)) = encode_col8(v, l, s2);
-}
-
-__device__ __forceinline__ void put_col_codes(uint8_t* row, const uint4 (&v)[4], int l, float2 s2,
-                                              int i, int j) {
-  *reinterpret_cast<uint32_t*>(row + ((i ^ (2 * j)) << 2)) = encode_col4(v, l, s2);
+// Magnitude maximum of two BF16 pairs, half by half, with the float
+// max-of-absolute-values instruction on the raw words: the result's halves
+// hold the larger |.| (its sign bits are the xor of the inputs' and are
+// cleared once at the end).  Measured 0.36 fewer instructions per element
+// than masking every word and taking integer maxima (the order of
+// non-negative BF16 values is the order of their bits, so both give the same
+// amax; NaN inputs are outside the contract).
+__device__ __forceinline__ uint32_t amax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 // Larger of the two 16-bit halves.
@@ -164,17 +165,14 @@ __device__ __forceinline__ uint4 lds_v4(const uint8_t* p) {
   return *reinterpret_cast<const uint4*>(p);
 }
 
-// Row k's amax (BF16 bits) out of the row-pair words of row_amax, for a
+// Row k's amax (BF16 bits) out of the four row-pair words of row_amax, for a
 // lane-dependent k: byte permutes pick the half-word (a plain or selected
 // array index would be lowered to a local-memory round trip).
-template <int NQ>
-__device__ __forceinline__ uint32_t pick_row_amax(const uint32_t (&rm)[NQ], int k) {
-  static_assert(NQ == 2 || NQ == 4, "2 or 4 row-pair words");
+__device__ __forceinline__ uint32_t pick_row_half(const uint32_t (&rm)[4], int k) {
   const uint32_t b = 2u * static_cast<uint32_t>(k & 3);  // byte of the half within a word pair
   const uint32_t sel = b | ((b + 1u) << 4);
-  uint32_t w = __byte_perm(rm[0], rm[1], sel);
-  if constexpr (NQ == 4) w = (k & 4) ? __byte_perm(rm[2], rm[3], sel) : w;
-  return w & 0xFFFFu;
+  const uint32_t lo = __byte_perm(rm[0], rm[1], sel), hi = __byte_perm(rm[2], rm[3], sel);
+  return ((k & 4) ? hi : lo) & 0xFFFFu;
 }
 
 // Byte offset, inside one 512-byte chunk of a blocked scale array, of the
@@ -183,11 +181,35 @@ __device__ __forceinline__ uint32_t blocked_in_chunk(int r) {
   return static_cast<uint32_t>((r & 31) * 16 + ((r >> 5) & 3) * 4);
 }
 
+// The transposed codes of tile (r0, c0), staged in qt_s, to global memory:
+// thread (c_base, part) writes 16 rows' codes (one 16-byte unit) of four
+// transposed rows.  Row c of the staged tile holds the 8-byte chunk of rows
+// 8i..8i+7 at position i ^ 2(c/8 & 7), so 16-byte unit u of row c is at
+// position u ^ (c/8 & 7).  Units that start past the last row are skipped
+// (the units that are written cover rows up to the next multiple of 16; rows
+// past the end read zeros, whose codes are 0, the padding the layout wants).
+__device__ __forceinline__ void qt_readout(const QuantParams& p, const uint8_t* qt_s, int32_t r0,
+                                           int32_t c0, int tid) {
+  const int c_base = tid >> 3, part = tid & 7;
+  if (r0 + 16 * part >= p.rows) return;
+  uint8_t* dst = p.qt + (int64_t)(c0 + c_base) * p.ld_qt + (r0 + 16 * part);
+  const int64_t pass_stride = (int64_t)32 * p.ld_qt;
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int c = pass * 32 + c_base;
+    const int unit = part ^ ((c >> 3) & 7);
+    *reinterpret_cast<uint4*>(dst) = lds_v4(qt_s + c * 128 + (unit << 4));
+    dst += pass_stride;
+  }
+}
+
 // RSHFL selects how the row scales reach the threads (ROW without BLOCK):
-// one thread per row derives the exponent and the 16 threads of the row read
-// it with shuffles (fewer ALU instructions: faster when each CTA has only a
-// few tiles), or all 16 derive it themselves (no cross-lane latency on the
-// encode path: faster on long tile streams).  Both give identical results.
+// the 16 lanes of a row group reduce-scatter the row maxima, one lane per row
+// derives the exponent and the others read 2^-e with shuffles (fewer
+// instructions: faster when each CTA has only a few tiles), or every lane
+// gets every row's amax by a butterfly and derives the exponents of its 8
+// rows itself, two rows per word (no cross-lane latency on the encode path:
+// faster on long tile streams).  Both give identical results.
 //
 // Addressing is kept out of the per-element work: every output pointer is
 // formed once per tile from per-thread constants and advanced by its stride,
@@ -195,16 +217,13 @@ __device__ __forceinline__ uint32_t blocked_in_chunk(int r) {
 template <bool ROW, bool COL, bool BLOCK, bool RSHFL>
 __global__ void __launch_bounds__(kQThreads, 2)
     quant_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantParams p) {
-  constexpr uint32_t kMag = 0x7FFF7FFFu;
   constexpr int kWarps = kQThreads / 32;
-  constexpr int RPT = kQRpt;
-  constexpr int kColsPerPass = kQThreads / 8;  // transposed rows copied out per pass
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;                                    // kQStages x 32 KB
-  uint8_t* qt_s = smem + kQStages * kQTileBytes;            // 16 KB transposed codes
-  uint32_t* col_part = reinterpret_cast<uint32_t*>(qt_s + 128 * 128);  // [8 warps][16][4]
+  uint8_t* qt_buf = smem + kQStages * kQTileBytes;          // 2 x 16 KB transposed codes
+  uint32_t* col_part = reinterpret_cast<uint32_t*>(qt_buf + 2 * kQtTileBytes);  // [8 warps][16][4]
   float* col_scale = reinterpret_cast<float*>(col_part + kWarps * 64);  // [128] 2^-e per column
   uint32_t* blk_part = reinterpret_cast<uint32_t*>(col_scale + 128);    // [8]
   uint64_t* full = reinterpret_cast<uint64_t*>(blk_part + kWarps);
@@ -256,92 +275,109 @@ __global__ void __launch_bounds__(kQThreads, 2)
     while (p_it < my_tiles && p_it < kQStages) issue_next();
 
   // per-thread constants of the output addressing
-  const uint32_t s_in_chunk = blocked_in_chunk(RPT * i + (j & (RPT - 1)));  // row scale byte (j < RPT)
-  const uint32_t s_half_chunk = blocked_in_chunk(RPT * i + (j >> 1));      // the same, row j >> 1
-  const uint32_t st_in_chunk = blocked_in_chunk(2 * (tid & 63));            // column scale bytes (tid < 64)
-  const int c_base = tid >> 3, part = tid & 7;                               // transposed readout
-  const int64_t qt_pass_stride = (int64_t)kColsPerPass * p.ld_qt;
-  // 4 rows per thread: the readout's 16-byte unit has its 8-byte halves
-  // swapped for odd column groups, the same parity in every pass
-  // (kColsPerPass is a multiple of 16)
-  const bool swap_halves = RPT == 4 && ((c_base >> 3) & 1);
+  const uint32_t s_own_row = blocked_in_chunk(8 * i + (j & 7));    // row scale byte (j < 8)
+  const uint32_t s_half_chunk = blocked_in_chunk(8 * i + (j >> 1));  // the same, row j >> 1
+  const uint32_t st_in_chunk = blocked_in_chunk(2 * (tid & 63));     // column scale bytes (tid < 64)
 
   int32_t tr = (int32_t)blockIdx.x / p.tiles_c, tc = (int32_t)blockIdx.x % p.tiles_c;
+  int32_t prev_r0 = 0, prev_c0 = 0;  // the tile whose transposed codes wait in qt_buf
   for (int32_t it = 0; it < my_tiles; ++it) {
     const int32_t r0 = tr * 128, c0 = tc * 128;
     const int s = it % kQStages;
     const bool ok = mbar_wait(&full[s], (uint32_t)((it / kQStages) & 1), abort_flag);
-    // this thread's RPT rows x 8 columns; rows past the end were filled with 0
-    uint4 v[RPT];
-    const uint8_t* tile = tiles + s * kQTileBytes + (RPT * i) * 256 + 16 * j;
+    // this thread's 8 rows x 8 columns; rows past the end were filled with 0
+    uint4 v[8];
+    const uint8_t* tile = tiles + s * kQTileBytes + (8 * i) * 256 + 16 * j;
 #pragma unroll
-    for (int k = 0; k < RPT; ++k) v[k] = ok ? lds_v4(tile + k * 256) : make_uint4(0, 0, 0, 0);
-    // every thread holds its part: stage s is free again (and if any wait gave
-    // up, the whole block stops here together)
+    for (int k = 0; k < 8; ++k) v[k] = ok ? lds_v4(tile + k * 256) : make_uint4(0, 0, 0, 0);
+    // every thread holds its part: stage s is free again, and every thread
+    // has finished the previous tile, its transposed codes included (and if
+    // any wait gave up, the whole block stops here together)
     if (__syncthreads_or(!ok)) break;
     if (tid == 0 && p_it < my_tiles) issue_next();
+    if (COL && it > 0) qt_readout(p, qt_buf + ((it - 1) & 1) * kQtTileBytes, prev_r0, prev_c0, tid);
 
     // ---- magnitudes: per-row amax of this thread's 8 columns (two rows per
-    // word) and per-column-pair amax of its 8 rows, from the same masked words
-    uint32_t rowmax[RPT / 2];
+    // word) and per-column-pair amax of its 8 rows
+    uint32_t rowmax[4];
+    uint32_t cm[4];
 #pragma unroll
-    for (int q = 0; q < RPT / 2; ++q) rowmax[q] = 0u;
-    uint32_t cm[4] = {0u, 0u, 0u, 0u};
-    uint32_t even_row = 0u;  // (even, odd)-column maxima of the last even row
-#pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      const uint32_t a0 = v[k].x & kMag, a1 = v[k].y & kMag, a2 = v[k].z & kMag,
-                     a3 = v[k].w & kMag;
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t a0 = v[k].x, a1 = v[k].y, a2 = v[k].z, a3 = v[k].w;
       if (ROW || BLOCK) {
-        // two rows per word: the low halves of rows k-1, k side by side, the
-        // high halves side by side, and one packed max of the two
-        const uint32_t t = __vmaxu2(__vmaxu2(a0, a1), __vmaxu2(a2, a3));
-        if (k & 1)
-          rowmax[k >> 1] = __vmaxu2(__byte_perm(even_row, t, 0x5410), __byte_perm(even_row, t, 0x7632));
-        else
-          even_row = t;
+        const uint32_t t = amax2(amax2(a0, a1), amax2(a2, a3));
+        // rows k-1, k side by side: low halves in one word, high halves in another
+        if (k & 1) {
+          const uint32_t e = rowmax[k >> 1];
+          rowmax[k >> 1] = amax2(__byte_perm(e, t, 0x5410), __byte_perm(e, t, 0x7632));
+        } else {
+          rowmax[k >> 1] = t;
+        }
       }
       if (COL && !BLOCK) {
-        cm[0] = __vmaxu2(cm[0], a0);
-        cm[1] = __vmaxu2(cm[1], a1);
-        cm[2] = __vmaxu2(cm[2], a2);
-        cm[3] = __vmaxu2(cm[3], a3);
+        if (k == 0) {
+          cm[0] = a0; cm[1] = a1; cm[2] = a2; cm[3] = a3;
+        } else {
+          cm[0] = amax2(cm[0], a0);
+          cm[1] = amax2(cm[1], a1);
+          cm[2] = amax2(cm[2], a2);
+          cm[3] = amax2(cm[3], a3);
+        }
       }
     }
-    // Row reductions over the 16 lanes of a row group.  On the shared-scale
-    // path with 8 rows per thread this is a reduce-scatter (rs_row below);
-    // elsewhere every lane needs every row's amax: a full butterfly.
-    constexpr bool kRowScatter = ROW && !BLOCK && RSHFL && RPT == 8;
-    if ((ROW || BLOCK) && !kRowScatter) {
 #pragma unroll
-      for (int q = 0; q < RPT / 2; ++q) {
+    for (int q = 0; q < 4; ++q) {
+      rowmax[q] &= 0x7FFF7FFFu;
+      if (COL && !BLOCK) cm[q] &= 0x7FFF7FFFu;
+    }
+
+    // ---- partial maxima for the block-wide reductions, then one barrier
+    if (COL && !BLOCK) {
 #pragma unroll
-        for (int off = 8; off >= 1; off >>= 1)
-          rowmax[q] = __vmaxu2(rowmax[q], __shfl_xor_sync(0xFFFFFFFFu, rowmax[q], off));
-      }
+      for (int pp = 0; pp < 4; ++pp)
+        cm[pp] = __vmaxu2(cm[pp], __shfl_xor_sync(0xFFFFFFFFu, cm[pp], 16));
+      if ((tid & 16) == 0)
+        *reinterpret_cast<uint4*>(&col_part[(warp * 16 + j) * 4]) = make_uint4(cm[0], cm[1], cm[2], cm[3]);
+    }
+    if (BLOCK) {
+      uint32_t m = __vmaxu2(__vmaxu2(rowmax[0], rowmax[1]), __vmaxu2(rowmax[2], rowmax[3]));
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+      if ((tid & 31) == 0) blk_part[warp] = hmax(m);
+    }
+    if ((COL && !BLOCK) || BLOCK) __syncthreads();
+
+    // ---- column scales: threads 0..63 reduce columns 2t, 2t+1 over the 8
+    // warps, store the two scale bytes and 2^-e for the encoders (published
+    // by the next barrier; meanwhile the other warps encode their rows)
+    if (COL && !BLOCK && tid < 64) {
+      uint32_t m = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) m = __vmaxu2(m, col_part[(w * 16 + (tid >> 2)) * 4 + (tid & 3)]);
+      const uint32_t k2 = scale_k2(m);
+      const uint32_t b2 = scale_bytes2(m, k2);
+      uint8_t* scol = p.st + ((int64_t)tc * p.st_g4 + (tr >> 2)) * 512 + (tr & 3) + st_in_chunk;
+      scol[0] = static_cast<uint8_t>(b2);
+      scol[16] = static_cast<uint8_t>(b2 >> 16);
+      *reinterpret_cast<float2*>(&col_scale[2 * tid]) = make_float2(scale_lo(k2), scale_hi(k2));
     }
 
     int e_blk = 0;
     if (BLOCK) {
-      // one exponent for the whole 128x128 block
-      uint32_t m = rowmax[0];
-#pragma unroll
-      for (int q = 1; q < RPT / 2; ++q) m = __vmaxu2(m, rowmax[q]);
-      m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
-      if ((tid & 31) == 0) blk_part[warp] = hmax(m);
-      __syncthreads();
       uint32_t bm = 0;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) bm = max(bm, blk_part[w]);
-      e_blk = scale_exponent_from_bits(bm);
+      const uint32_t k = scale_k2(bm) & 0xFFFFu;
+      e_blk = 127 - (int)k;
+      if (bm == 0) e_blk = 0;
       if (tid == 0) p.sw[tr * p.tiles_c + tc] = static_cast<uint8_t>(e_blk + 127);
     }
 
-    // ---- in-place codes (ROW, BLOCK) and the row scale bytes; thread j < RPT
-    // owns the scale byte of row RPT*i + j
+    // ---- in-place codes (ROW, BLOCK) and the row scale bytes
     if (ROW || BLOCK) {
-      uint8_t* qrow = p.q + (int64_t)(r0 + RPT * i) * p.ld_q + (c0 + 8 * j);
-      const int32_t nrow = (int32_t)(p.rows - r0) - RPT * i;  // rows of the block that exist
+      uint8_t* qrow = p.q + (int64_t)(r0 + 8 * i) * p.ld_q + (c0 + 8 * j);
+      const int32_t nrow = (int32_t)(p.rows - r0) - 8 * i;  // rows of the block that exist
+      constexpr bool kRowScatter = ROW && !BLOCK && RSHFL;
       if (kRowScatter) {
         // Reduce-scatter of the four row-pair words over the 16 lanes (lane
         // bits b3 b2 b1 b0 = j): at distance 8 a lane keeps the pair of words
@@ -359,45 +395,47 @@ __global__ void __launch_bounds__(kQThreads, 2)
         w = __vmaxu2(w, __shfl_xor_sync(0xFFFFFFFFu, b2 ? k0 : k1, 4));
         w = __vmaxu2(w, __shfl_xor_sync(0xFFFFFFFFu, w, 2));
         w = __vmaxu2(w, __shfl_xor_sync(0xFFFFFFFFu, w, 1));
-        const int e_mine = scale_exponent_from_bits(b1 ? (w >> 16) : (w & 0xFFFFu));
+        const uint32_t k2 = scale_k2(w);
+        const uint32_t bytes = scale_bytes2(w, k2);
         if ((j & 1) == 0)
-          p.s[((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_half_chunk] = static_cast<uint8_t>(e_mine + 127);
-        const float s_mine = pow2_neg_x2(e_mine).x;
+          p.s[((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_half_chunk] =
+              static_cast<uint8_t>(b1 ? (bytes >> 16) : bytes);
+        const float s_mine = b1 ? scale_hi(k2) : scale_lo(k2);
         const int lane16 = tid & 16;
 #pragma unroll
-        for (int k = 0; k < RPT; ++k) {
+        for (int k = 0; k < 8; ++k) {
           const float sk = __shfl_sync(0xFFFFFFFFu, s_mine, lane16 + 2 * k);
           const uint2 o = encode_row8(v[k], make_float2(sk, sk));
           if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
           qrow += p.ld_q;
         }
-      } else if (RSHFL && !BLOCK) {
-        // thread j derives row RPT*i + j's exponent; the 16 threads of the
-        // rows read 2^-e of row k from thread k
-        const int e_mine = scale_exponent_from_bits(pick_row_amax(rowmax, j & (RPT - 1)));
-        if (j < RPT)
-          p.s[((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_in_chunk] = static_cast<uint8_t>(e_mine + 127);
-        const float s_mine = pow2_neg_x2(e_mine).x;
-        const int lane16 = tid & 16;
-#pragma unroll
-        for (int k = 0; k < RPT; ++k) {
-          const float sk = __shfl_sync(0xFFFFFFFFu, s_mine, lane16 + k);
-          const uint2 o = encode_row8(v[k], make_float2(sk, sk));
-          if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
-          qrow += p.ld_q;
-        }
       } else {
-        // every thread derives the exponents of its rows itself (the scale
-        // byte is stored inside the loop, its address formed there: deriving
-        // the byte ahead of the encodes, or keeping its pointer live across
-        // the loop, was measured 10 % slower on long tile streams)
+        // every lane gets every row's amax (butterfly) and derives its 8 rows'
+        // exponents two at a time; lane j < 8 stores row 8i + j's scale byte
+        float sc[8];
+        if (BLOCK) {
+          const float f = __uint_as_float(static_cast<uint32_t>(127 - e_blk) << 23);
 #pragma unroll
-        for (int k = 0; k < RPT; ++k) {
-          const uint32_t m = (k & 1) ? (rowmax[k >> 1] >> 16) : (rowmax[k >> 1] & 0xFFFFu);
-          const int e = BLOCK ? e_blk : scale_exponent_from_bits(m);
-          const uint2 o = encode_row8(v[k], pow2_neg_x2(e));
-          if (!BLOCK && j == k)
-            p.s[((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_in_chunk] = static_cast<uint8_t>(e + 127);
+          for (int k = 0; k < 8; ++k) sc[k] = f;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+#pragma unroll
+            for (int off = 8; off >= 1; off >>= 1)
+              rowmax[q] = __vmaxu2(rowmax[q], __shfl_xor_sync(0xFFFFFFFFu, rowmax[q], off));
+            const uint32_t k2 = scale_k2(rowmax[q]);
+            sc[2 * q] = scale_lo(k2);
+            sc[2 * q + 1] = scale_hi(k2);
+          }
+          if (j < 8) {
+            const uint32_t a = pick_row_half(rowmax, j);
+            const uint32_t b = scale_bytes2(a, scale_k2(a)) & 0xFFu;
+            p.s[((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_own_row] = static_cast<uint8_t>(b);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint2 o = encode_row8(v[k], make_float2(sc[k], sc[k]));
           if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
           qrow += p.ld_q;
         }
@@ -406,58 +444,29 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
     // ---- transposed codes (COL, BLOCK with a transposed copy)
     if (COL) {
-      if (!BLOCK) {
-#pragma unroll
-        for (int pp = 0; pp < 4; ++pp)
-          cm[pp] = __vmaxu2(cm[pp], __shfl_xor_sync(0xFFFFFFFFu, cm[pp], 16));
-        if ((tid & 16) == 0)
-          *reinterpret_cast<uint4*>(&col_part[(warp * 16 + j) * 4]) = make_uint4(cm[0], cm[1], cm[2], cm[3]);
-        __syncthreads();
-        if (tid < 64) {
-          // columns 2*tid and 2*tid+1: amax over the 8 warps, then the exponent,
-          // its scale byte and 2^-e for every thread's encode
-          uint32_t m = 0;
-#pragma unroll
-          for (int w = 0; w < kWarps; ++w) m = __vmaxu2(m, col_part[(w * 16 + (tid >> 2)) * 4 + (tid & 3)]);
-          const int e0 = scale_exponent_from_bits(m & 0xFFFFu);
-          const int e1 = scale_exponent_from_bits(m >> 16);
-          uint8_t* scol = p.st + ((int64_t)tc * p.st_g4 + (tr >> 2)) * 512 + (tr & 3) + st_in_chunk;
-          scol[0] = static_cast<uint8_t>(e0 + 127);
-          scol[16] = static_cast<uint8_t>(e1 + 127);
-          *reinterpret_cast<float2*>(&col_scale[2 * tid]) = make_float2(pow2_neg_x2(e0).x, pow2_neg_x2(e1).x);
-        }
-        __syncthreads();
-      }
+      if (!BLOCK) __syncthreads();   // column scales published
       float cs[8];
-      if (!BLOCK) {
+      if (BLOCK) {
+        const float f = __uint_as_float(static_cast<uint32_t>(127 - e_blk) << 23);
+#pragma unroll
+        for (int l = 0; l < 8; ++l) cs[l] = f;
+      } else {
         const float4 a = *reinterpret_cast<const float4*>(&col_scale[8 * j]);
         const float4 b = *reinterpret_cast<const float4*>(&col_scale[8 * j + 4]);
         cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
         cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
       }
+      uint8_t* qt_s = qt_buf + (it & 1) * kQtTileBytes;
+      // row (8j+l) of the transposed tile: this thread's 8 codes go to 8-byte
+      // chunk i ^ 2(j & 7), so that a 16-byte unit holds two consecutive
+      // chunks in order while the 32 stores of a warp fill 16 distinct chunk
+      // positions twice (two wavefronts, the minimum for 256 bytes)
+      uint8_t* dst = qt_s + (8 * j) * 128 + ((i ^ (2 * (j & 7))) << 3);
 #pragma unroll
-      for (int l = 0; l < 8; ++l) {
-        const float2 s2 = BLOCK ? pow2_neg_x2(e_blk) : make_float2(cs[l], cs[l]);
-        // row (8j+l) of the transposed tile: this thread's RPT codes go to an
-        // XOR-swizzled chunk (put_col_codes) that the readout below undoes
-        put_col_codes(qt_s + (8 * j + l) * 128, v, l, s2, i, j);
-      }
-      __syncthreads();
-      // transposed row c = pass * kColsPerPass + c_base, rows 16*part.. of the
-      // tile: with jj = c / 8 its 16 codes sit in 16-byte unit part ^ (jj & 7)
-      // (8 rows per thread) or part ^ (jj >> 1) (4 rows per thread)
-      if (r0 + 16 * part < p.rows) {
-        uint8_t* dst = p.qt + (int64_t)(c0 + c_base) * p.ld_qt + (r0 + 16 * part);
-#pragma unroll
-        for (int pass = 0; pass < 128 / kColsPerPass; ++pass) {
-          const int c = pass * kColsPerPass + c_base;
-          const int unit = part ^ (RPT == 8 ? ((c >> 3) & 7) : ((c >> 4) & 7));
-          uint4 w = lds_v4(qt_s + c * 128 + (unit << 4));
-          if (swap_halves) w = make_uint4(w.z, w.w, w.x, w.y);
-          *reinterpret_cast<uint4*>(dst) = w;
-          dst += qt_pass_stride;
-        }
-      }
+      for (int l = 0; l < 8; ++l)
+        *reinterpret_cast<uint2*>(dst + l * 128) = encode_col8(v, l, make_float2(cs[l], cs[l]));
+      prev_r0 = r0;
+      prev_c0 = c0;
     }
 
     if (BLOCK && tid < 128) {
@@ -466,12 +475,18 @@ __global__ void __launch_bounds__(kQThreads, 2)
       if (p.sw_fwd) p.sw_fwd[((int64_t)tr * p.fwd_g4 + (tc >> 2)) * 512 + (tc & 3) + in_chunk] = b;
       if (p.sw_bwd) p.sw_bwd[((int64_t)tc * p.bwd_g4 + (tr >> 2)) * 512 + (tr & 3) + in_chunk] = b;
     }
-    // No barrier here: the shared tiles (qt_s, col_part, blk_part) are next
-    // written after the __syncthreads_or at the top of the next iteration,
-    // which no thread passes before every thread has finished this tile.
+    // No barrier here: the shared tiles (col_part, col_scale, blk_part, the
+    // other transposed buffer) are next written after the barrier at the top
+    // of the next iteration, which no thread passes before every thread has
+    // finished this tile.
     tc += tc_step;
     tr += tr_step;
     if (tc >= p.tiles_c) { tc -= p.tiles_c; ++tr; }
+  }
+  // the last tile's transposed codes (if every wait succeeded)
+  if (COL && my_tiles > 0) {
+    if (!__syncthreads_or(*abort_flag != 0))
+      qt_readout(p, qt_buf + ((my_tiles - 1) & 1) * kQtTileBytes, prev_r0, prev_c0, tid);
   }
   // Copies are only issued for tiles this CTA processes, and each one was
   // waited for above, unless a wait gave up; then let the outstanding ones
@@ -487,7 +502,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
 // Shared memory the quantizer needs (plus alignment slack).
 constexpr uint32_t quant_smem_bytes() {
-  return kQStages * kQTileBytes + 128 * 128 + (kQThreads / 32) * 64 * 4 + 128 * 4 +
+  return kQStages * kQTileBytes + 2 * kQtTileBytes + (kQThreads / 32) * 64 * 4 + 128 * 4 +
          (kQThreads / 32) * 4 + kQStages * 8 + 16 + 1024;
 }
 

@@ -77,9 +77,25 @@ struct GemmProblem {
   int32_t rows_b;      // output cols
   int32_t kblocks;     // ceil(K / BK)
   int32_t tiles_m, tiles_n;
+  int32_t n_fastest;   // tile t -> (t / tiles_n, t % tiles_n) instead of (t % tiles_m, t / tiles_m)
   int32_t split_from;  // first split tile (== tiles_m * tiles_n: none)
   int32_t units;       // split_from + 2 * (tiles - split_from)
 };
+
+// Row and column tile of tile index t.  Consecutive tiles run at the same
+// time on consecutive clusters, so the operand whose tiles are shared by
+// consecutive indices is the one L2 keeps: with n_fastest they share A's rows
+// (the host sets it when A is the larger operand, e.g. the activations of a
+// forward or data-gradient GEMM with many tokens); otherwise they share B's.
+__device__ __forceinline__ void tile_coords(const GemmProblem& P, int t, int& tm, int& tn) {
+  if (P.n_fastest) {
+    tm = t / P.tiles_n;
+    tn = t - tm * P.tiles_n;
+  } else {
+    tn = t / P.tiles_m;
+    tm = t - tn * P.tiles_m;
+  }
+}
 
 // Tile and half (-1: whole tile, 0/1: left/right half) of a problem's unit.
 __device__ __forceinline__ void decode_unit(const GemmProblem& P, int lu, int& tile, int& h) {
@@ -341,7 +357,8 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       const CUtensorMap* tm_b = halft ? (pr ? &tm_bh1 : &tm_bh0) : (pr ? &tm_b1 : &tm_b0);
       const CUtensorMap* tm_sfa = pr ? &tm_sfa1 : &tm_sfa0;
       const CUtensorMap* tm_sfb = pr ? &tm_sfb1 : &tm_sfb0;
-      const int tm = tile % P.tiles_m, tn = tile / P.tiles_m;
+      int tm, tn;
+      tile_coords(P, tile, tm, tn);
       const int a_row = tm * C::kBM + 128 * (int)rank;
       const int b_col0 = tn * BN + (halft ? (BN / 2) * h : 0);   // first output column
       const int b_row = b_col0 + (halft ? C::kBNC / 2 : C::kBNC) * (int)rank;
@@ -461,7 +478,8 @@ __global__ void __launch_bounds__(GemmCfg<CG, BN, BK>::kThreads, 1)
       const GemmProblem& P = p.prob[pr];
       int tile, h;
       decode_unit(P, u - (pr ? p.tiles0 : 0), tile, h);
-      const int tm = tile % P.tiles_m, tn = tile / P.tiles_m;
+      int tm, tn;
+      tile_coords(P, tile, tm, tn);
       const int acc = it % NA;
       const uint32_t acc_phase = (it / NA) & 1;
       if (!mbar_wait(&accf[acc], acc_phase, abort_flag)) break;

@@ -294,6 +294,9 @@ int launch_gemm_cfg(const GemmArgs& g0, const GemmArgs* g1, DeviceInfo* dev, cud
     p.prob[i].kblocks = (int32_t)((g.k + BK - 1) / BK);
     p.prob[i].tiles_m = (int32_t)((g.rows_a + C::kBM - 1) / C::kBM);
     p.prob[i].tiles_n = (int32_t)((g.rows_b + BN - 1) / BN);
+    // the larger operand is walked in the slower index, so that the tiles
+    // running at the same time share its rows and L2 keeps them
+    p.prob[i].n_fastest = g.rows_a > g.rows_b ? 1 : 0;
   }
   const int C_max = max_clusters[dev_id].load(std::memory_order_acquire);
   for (int i = 0; i < p.nprob; ++i) {

@@ -104,3 +104,18 @@ def test_mfu_accounting_closed_forms():
     out = bench.mfu_accounting(1800.0, 1270.0, peaks)
     assert math.isclose(out["projected_tflops"], 1611.7, abs_tol=0.05)
     assert math.isclose(out["mfu_vs_measured"], 0.7368, abs_tol=1e-4)
+
+
+def test_gemm_peak_regime():
+    # a short run at full clock: the burst peak
+    assert bench.gemm_peak({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}, 3180.0, 2800.0) == (
+        3180.0, "burst")
+    # power cap active but the clock held up: still burst
+    assert bench.gemm_peak({"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]},
+                           3180.0, 2800.0)[1] == "burst"
+    # a long power-capped run at 1.1 GHz: the sustained peak
+    assert bench.gemm_peak({"sm_mhz": 1100.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]},
+                           3180.0, 2800.0) == (2800.0, "sustained")
+    # no clock record: burst
+    assert bench.gemm_peak({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]},
+                           3180.0, 2800.0)[1] == "burst"

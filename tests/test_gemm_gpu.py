@@ -45,6 +45,8 @@ def _run(fp8, x, w, dy):
     (129, 256, 384),
     (520, 640, 256),     # N not a multiple of the 256-wide tile
     (64, 128, 1024),
+    (1300, 768, 640),    # several tiles both ways, tiles walked along N (A is larger)
+    (300, 1280, 768),    # several tiles both ways, tiles walked along M (B is larger)
 ])
 def test_linear_layer_small(fp8, oracle_mod, m, n, k):
     x, w, dy = _layer(m, n, k, m + n + k)

@@ -34,10 +34,10 @@
 // and the order of non-negative floats equals the order of their bits), and
 // the scale exponent comes from the exponent/mantissa fields alone, two
 // groups per 32-bit word: with amax = 1.f * 2^E, e = E - 8 if 1.f <= 1.75
-// (mantissa bits <= 0x60), else E - 7.  Scaling by 2^-e is an exact packed
-// FP32 multiply (no flush to zero: this file must not be built with
-// fast-math), followed by one hardware round-to-nearest-even, saturating
-// conversion to E4M3 per value.
+// (mantissa bits <= 0x60), else E - 7.  Scaling by 2^-e is an exact
+// BF16 x BF16 -> FP32 fused multiply-add (no flush to zero: this file must
+// not be built with fast-math), followed by one hardware round-to-nearest-even,
+// saturating conversion to E4M3 per value.
 #pragma once
 
 #include "common.cuh"
@@ -95,53 +95,98 @@ __device__ __forceinline__ uint32_t scale_bytes2(uint32_t a2, uint32_t k2) {
 __device__ __forceinline__ float scale_lo(uint32_t k2) { return __uint_as_float(k2 << 23); }
 __device__ __forceinline__ float scale_hi(uint32_t k2) { return __uint_as_float((k2 << 7) & 0x7F800000u); }
 
-// Four values (pairs a, b) times 2^-e (s2) -> four E4M3 codes in one word,
-// a.x in the low byte.  The packed multiply is exact (a power of two,
-// subnormals kept), then one RNE saturating conversion per value; the two
-// 16-bit results are joined by a register move rather than shift-and-or
-// (measured: 8 fewer ALU instructions per 32 values on sm_100a).
-__device__ __forceinline__ uint32_t encode4(float2 a, float2 b, float2 s2) {
-  const float2 x = __fmul2_rn(a, s2), y = __fmul2_rn(b, s2);
+// 2^-e as BF16 bits, from its FP32 form (exact: a power of two with e in
+// [-127, 120] is a normal BF16).
+__device__ __forceinline__ uint16_t bf16_bits(float f) {
+  return static_cast<uint16_t>(__float_as_uint(f) >> 16);
+}
+
+// Encoding x * 2^-e to E4M3: fma.rn.f32.bf16 forms the product of the BF16
+// value and the BF16 scale exactly in FP32 (two 8-bit significands fit in
+// FP32's 24; subnormals kept) and adds -0.0, which leaves every value and the
+// sign of zero unchanged; then one round-to-nearest-even, saturating
+// conversion per value.  Taking the BF16 operand straight from a half of the
+// loaded word saves the separate widening to FP32 (measured: one instruction
+// per element less than widening and a packed FP32 multiply); the codes are
+// the same for every BF16 value and every scale (checked exhaustively).
+// The two 16-bit results are joined by a register move.
+
+// Four codes of the BF16 pairs w01 = (x0, x1) and w23 = (x2, x3), x0 in the
+// low byte.
+__device__ __forceinline__ uint32_t encode4_pairs(uint32_t w01, uint32_t w23, uint16_t s) {
   uint32_t r;
-  asm("{\n\t.reg .b16 lo, hi;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+  asm("{\n\t.reg .b16 a0, a1, b0, b1, lo, hi;\n\t.reg .f32 f0, f1, f2, f3;\n\t"
+      "mov.b32 {a0, a1}, %1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.bf16 f0, a0, %3, 0f80000000;\n\t"
+      "fma.rn.f32.bf16 f1, a1, %3, 0f80000000;\n\t"
+      "fma.rn.f32.bf16 f2, b0, %3, 0f80000000;\n\t"
+      "fma.rn.f32.bf16 f3, b1, %3, 0f80000000;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, f1, f0;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, f3, f2;\n\t"
       "mov.b32 %0, {lo, hi};\n\t}"
       : "=r"(r)
-      : "f"(x.x), "f"(x.y), "f"(y.x), "f"(y.y));
+      : "r"(w01), "r"(w23), "h"(s));
   return r;
 }
 
-// The two BF16 of a packed word widened to FP32 (exact).
-__device__ __forceinline__ float2 bf16x2_f32(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+// Four codes of one half (H = 0: low, 1: high) of the words w0..w3 -- one
+// column of four consecutive rows -- w0's in the low byte.
+template <int H>
+__device__ __forceinline__ uint32_t encode4_col(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                                uint16_t s) {
+  uint32_t r;
+  if (H == 0)
+    asm("{\n\t.reg .b16 x0, x1, x2, x3, y0, y1, y2, y3, lo, hi;\n\t.reg .f32 f0, f1, f2, f3;\n\t"
+        "mov.b32 {x0, y0}, %1;\n\t"
+        "mov.b32 {x1, y1}, %2;\n\t"
+        "mov.b32 {x2, y2}, %3;\n\t"
+        "mov.b32 {x3, y3}, %4;\n\t"
+        "fma.rn.f32.bf16 f0, x0, %5, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 f1, x1, %5, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 f2, x2, %5, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 f3, x3, %5, 0f80000000;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, f1, f0;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, f3, f2;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r)
+        : "r"(w0), "r"(w1), "r"(w2), "r"(w3), "h"(s));
+  else
+    asm("{\n\t.reg .b16 x0, x1, x2, x3, y0, y1, y2, y3, lo, hi;\n\t.reg .f32 f0, f1, f2, f3;\n\t"
+        "mov.b32 {y0, x0}, %1;\n\t"
+        "mov.b32 {y1, x1}, %2;\n\t"
+        "mov.b32 {y2, x2}, %3;\n\t"
+        "mov.b32 {y3, x3}, %4;\n\t"
+        "fma.rn.f32.bf16 f0, x0, %5, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 f1, x1, %5, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 f2, x2, %5, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 f3, x3, %5, 0f80000000;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, f1, f0;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, f3, f2;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r)
+        : "r"(w0), "r"(w1), "r"(w2), "r"(w3), "h"(s));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t word(const uint4& v, int idx) {
   return idx == 0 ? v.x : idx == 1 ? v.y : idx == 2 ? v.z : v.w;
 }
 
-// Element l (0..7) of an 8-BF16 row chunk, widened to FP32.
-__device__ __forceinline__ float elem_f32(const uint4& v, int l) {
-  const uint32_t w = word(v, l >> 1);
-  return __uint_as_float((l & 1) ? (w & 0xFFFF0000u) : (w << 16));
-}
-
-// Eight codes of one 8-element row chunk, all scaled by s2.
-__device__ __forceinline__ uint2 encode_row8(const uint4& v, float2 s2) {
+// Eight codes of one 8-element row chunk, all scaled by 2^-e (BF16 bits s).
+__device__ __forceinline__ uint2 encode_row8(const uint4& v, uint16_t s) {
   uint2 o;
-  o.x = encode4(bf16x2_f32(v.x), bf16x2_f32(v.y), s2);
-  o.y = encode4(bf16x2_f32(v.z), bf16x2_f32(v.w), s2);
+  o.x = encode4_pairs(v.x, v.y, s);
+  o.y = encode4_pairs(v.z, v.w, s);
   return o;
 }
 
-// Eight codes of column l of the thread's 8x8 block (rows 0..7), scaled by s2.
-__device__ __forceinline__ uint2 encode_col8(const uint4 (&v)[8], int l, float2 s2) {
+// Eight codes of column l of the thread's 8x8 block (rows 0..7), scaled by s.
+template <int L>
+__device__ __forceinline__ uint2 encode_col8(const uint4 (&v)[8], uint16_t s) {
   uint2 o;
-  o.x = encode4(make_float2(elem_f32(v[0], l), elem_f32(v[1], l)),
-                make_float2(elem_f32(v[2], l), elem_f32(v[3], l)), s2);
-  o.y = encode4(make_float2(elem_f32(v[4], l), elem_f32(v[5], l)),
-                make_float2(elem_f32(v[6], l), elem_f32(v[7], l)), s2);
+  o.x = encode4_col<L & 1>(word(v[0], L >> 1), word(v[1], L >> 1), word(v[2], L >> 1), word(v[3], L >> 1), s);
+  o.y = encode4_col<L & 1>(word(v[4], L >> 1), word(v[5], L >> 1), word(v[6], L >> 1), word(v[7], L >> 1), s);
   return o;
 }
 
@@ -405,7 +450,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const float sk = __shfl_sync(0xFFFFFFFFu, s_mine, lane16 + 2 * k);
-          const uint2 o = encode_row8(v[k], make_float2(sk, sk));
+          const uint2 o = encode_row8(v[k], bf16_bits(sk));
           if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
           qrow += p.ld_q;
         }
@@ -435,7 +480,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint2 o = encode_row8(v[k], make_float2(sc[k], sc[k]));
+          const uint2 o = encode_row8(v[k], bf16_bits(sc[k]));
           if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
           qrow += p.ld_q;
         }
@@ -462,9 +507,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
       // chunks in order while the 32 stores of a warp fill 16 distinct chunk
       // positions twice (two wavefronts, the minimum for 256 bytes)
       uint8_t* dst = qt_s + (8 * j) * 128 + ((i ^ (2 * (j & 7))) << 3);
-#pragma unroll
-      for (int l = 0; l < 8; ++l)
-        *reinterpret_cast<uint2*>(dst + l * 128) = encode_col8(v, l, make_float2(cs[l], cs[l]));
+      *reinterpret_cast<uint2*>(dst + 0 * 128) = encode_col8<0>(v, bf16_bits(cs[0]));
+      *reinterpret_cast<uint2*>(dst + 1 * 128) = encode_col8<1>(v, bf16_bits(cs[1]));
+      *reinterpret_cast<uint2*>(dst + 2 * 128) = encode_col8<2>(v, bf16_bits(cs[2]));
+      *reinterpret_cast<uint2*>(dst + 3 * 128) = encode_col8<3>(v, bf16_bits(cs[3]));
+      *reinterpret_cast<uint2*>(dst + 4 * 128) = encode_col8<4>(v, bf16_bits(cs[4]));
+      *reinterpret_cast<uint2*>(dst + 5 * 128) = encode_col8<5>(v, bf16_bits(cs[5]));
+      *reinterpret_cast<uint2*>(dst + 6 * 128) = encode_col8<6>(v, bf16_bits(cs[6]));
+      *reinterpret_cast<uint2*>(dst + 7 * 128) = encode_col8<7>(v, bf16_bits(cs[7]));
       prev_r0 = r0;
       prev_c0 = c0;
     }

@@ -60,12 +60,28 @@ SPEC_FP8_TFLOPS = 4500.0     # B200 dense FP8 tensor-core peak (spec)
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
 SPEC_SM_MHZ = 1965.0         # B200 maximum SM clock, at which the spec peak is quoted
+LOADED_WATTS = 500.0         # board power above which a clock sample counts as under load
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch, from ncu captures
-# (one-pass metrics on the full-size default workload), keyed by launch name;
-# None when the kernel has changed since it was captured.
-GEMM_TRAFFIC_BYTES = None
-QUANT_TRAFFIC_BYTES = None
+# dram__bytes_read.sum + dram__bytes_write.sum of every launch of one step of
+# the default workload (full block, 32768 tokens), from a one-pass ncu capture
+# of the current kernels:
+#   ncu --clock-control none --metrics gpu__time_duration.sum,dram__bytes_read.sum,
+#       dram__bytes_write.sum -c 200 --csv python bench.py --steps 2 --warmup 1
+#       --accum 2 --no-sweep --no-e2e --no-cpu-baseline --no-ceiling --no-bf16
+# (serialised launches: each one starts with its inputs in DRAM, and what it
+# writes last may still sit in L2 when it ends).  To be emptied whenever a
+# kernel changes, until it is captured again.
+TRAFFIC_WORKLOAD = "full_block_m32768"
+TRAFFIC_BYTES = {
+    "qkv.quant_weight": 12_600_000, "qkv.quant_x": 211_800_000, "qkv.fprop": 222_000_000,
+    "qkv.quant_dy": 349_100_000, "qkv.dgrad_wgrad": 497_000_000,
+    "o_proj.quant_weight": 8_400_000, "o_proj.quant_x": 211_300_000, "o_proj.fprop": 156_200_000,
+    "o_proj.quant_dy": 212_100_000, "o_proj.dgrad_wgrad": 325_400_000,
+    "gate_up.quant_weight": 50_900_000, "gate_up.quant_x": 212_000_000, "gate_up.fprop": 887_900_000,
+    "gate_up.quant_dy": 1_577_400_000, "gate_up.dgrad_wgrad": 2_065_000_000,
+    "down.quant_weight": 25_200_000, "down.quant_x": 759_300_000, "down.fprop": 325_000_000,
+    "down.quant_dy": 211_900_000, "down.dgrad_wgrad": 995_200_000,
+}
 
 
 def _peaks():
@@ -190,11 +206,14 @@ def _num(s):
 def summarize_clocks(rows):
     """rows: nvidia-smi fields index, clocks.sm, clocks.max.sm, power.draw,
     utilization.gpu, hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown,
-    sw_power_cap.  Median SM clock over the loaded samples (all samples if
-    none is loaded); every throttle reason seen Active in a loaded sample."""
+    sw_power_cap.  A sample is under load when the utilisation reads >= 50 %
+    or the board draws >= LOADED_WATTS (the utilisation counter averages over
+    a longer window than the sampling period and lags behind a short run).
+    Median SM clock over the loaded samples (all samples if none is loaded);
+    every throttle reason seen Active in a loaded sample."""
     if not rows:
         return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-    loaded = [r for r in rows if (_num(r[4]) or 0.0) >= 50.0]
+    loaded = [r for r in rows if (_num(r[4]) or 0.0) >= 50.0 or (_num(r[3]) or 0.0) >= LOADED_WATTS]
     use = loaded or rows
     sm = [v for v in (_num(r[1]) for r in use) if v is not None]
     mx = [v for v in (_num(r[2]) for r in rows) if v is not None]
@@ -304,7 +323,9 @@ def _unit_costs(wl):
 def measure(wl, dev, world, K, warmup, accum, gpu, inst_steps=100):
     """Times K steps of the workload on the device (CUDA graphs of `accum`
     steps, the gradient exchange between them) and, separately, per-launch
-    times from an instrumented replay.  Returns the raw measurements."""
+    times from an instrumented replay of `inst_steps` steps (long enough for
+    the clock samples taken over both to catch the GPU under load).  Returns
+    the raw measurements."""
     import torch
     import torch.distributed as dist
 
@@ -328,7 +349,7 @@ def measure(wl, dev, world, K, warmup, accum, gpu, inst_steps=100):
     # event nodes between kernels also cut the programmatic (PDL) edges that
     # let a kernel's prologue overlap its predecessor's tail.
     windows = [A] * (K // A) + ([K % A] if K % A else [])
-    K_inst = min(K, inst_steps)
+    K_inst = inst_steps
     inst_names = [step.launch_names(i % A == 0) for i in range(K_inst)]
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * len(nm))]
           for nm in inst_names]
@@ -389,7 +410,7 @@ def measure(wl, dev, world, K, warmup, accum, gpu, inst_steps=100):
             "inst_steps": K_inst, "n_sets": n_sets}
 
 
-def summarize(wl, res, peaks, peak_kind, world):
+def summarize(wl, res, peaks, peak_kind, world, wl_tag=None):
     """value, GEMM roofline, quantizer roofline and per-kernel breakdown."""
     costs = _unit_costs(wl)
     gemm_flops = wl.gemm_flops()
@@ -405,12 +426,23 @@ def summarize(wl, res, peaks, peak_kind, world):
     act_names = [n for n in names if costs[n][0] == "bytes" and not n.endswith("quant_weight")]
     act_ms = sum(sum(pl[n]) for n in act_names)
     act_gbs = sum(costs[n][1] * len(pl[n]) for n in act_names) / (act_ms * 1e-3) / 1e9
+    traffic = TRAFFIC_BYTES if wl_tag == TRAFFIC_WORKLOAD else {}
     breakdown = {}
     for n in names:
         kind, amount = costs[n]
         ms = statistics.mean(pl[n])
         rate = amount / (ms * 1e-3) / (1e12 if kind == "flops" else 1e9)
         breakdown[n] = {"ms": round(ms, 5), ("tflops" if kind == "flops" else "gbs"): round(rate, 1)}
+        if n in traffic:
+            breakdown[n]["dram_bytes"] = traffic[n]
+            if kind == "bytes":
+                breakdown[n]["algorithmic_bytes"] = amount
+
+    def mean_traffic(which):
+        sel = [n for n in names if costs[n][0] == which]
+        if not traffic or any(n not in traffic for n in sel):
+            return None
+        return int(sum(traffic[n] for n in sel) / len(sel))
     burst = 2.0 * peaks["bf16_tflops"]
     sustained = 2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     peak, regime = gemm_peak(res["clocks"], burst, sustained)
@@ -434,7 +466,9 @@ def summarize(wl, res, peaks, peak_kind, world):
         "spec_peak": SPEC_FP8_TFLOPS,
         "frac_vs_spec_at_clock": (round(gemm_tf / (SPEC_FP8_TFLOPS * clk / SPEC_SM_MHZ), 4)
                                   if clk else None),
-        "traffic": GEMM_TRAFFIC_BYTES,
+        "traffic": mean_traffic("flops"),
+        "traffic_what": "DRAM bytes read + written per GEMM launch, averaged over the step's GEMM "
+                        "launches (per launch in `kernels`), from a one-pass ncu capture",
     }
     quant = {
         "bound": "hbm", "achieved": round(quant_gbs, 1), "unit": "GB/s",
@@ -443,7 +477,7 @@ def summarize(wl, res, peaks, peak_kind, world):
         "frac_vs_spec": round(quant_gbs / SPEC_HBM_GBS, 4), "spec_peak": SPEC_HBM_GBS,
         "activations_only": {"achieved": round(act_gbs, 1),
                              "frac": round(act_gbs / peaks["hbm_gbs"], 4)},
-        "traffic": QUANT_TRAFFIC_BYTES,
+        "traffic": mean_traffic("bytes"),
         "what": "every quantizer launch of the instrumented replay, algorithmic bytes over "
                 "per-launch event time (each launch timed on its own, without the overlap "
                 "with its neighbours that the timed graphs have)",
@@ -488,7 +522,7 @@ def run_ours(args):
     wl = make_workload(args.workload, args.m, seed_offset=rank)
     set_bytes = input_set_bytes(wl)
     res = measure(wl, dev, world, args.steps, args.warmup, args.accum, smi_id(local))
-    sm = summarize(wl, res, peaks, peak_kind, world)
+    sm = summarize(wl, res, peaks, peak_kind, world, workload_tag(args.workload, args.m))
     step = res["step"]
     A = res["accum"]
     gemm_flops = sm["gemm_flops"]
@@ -616,7 +650,7 @@ def run_sweep(args, dev, peaks, peak_kind):
         wl = make_workload(name, m)
         A = max(1, WINDOW_TOKENS // m)
         res = measure(wl, dev, 1, K, max(3, min(args.warmup, 5)), A, smi_id(dev.index))
-        sm = summarize(wl, res, peaks, peak_kind, 1)
+        sm = summarize(wl, res, peaks, peak_kind, 1, workload_tag(name, m))
         entry = {"ms_per_step": round(res["ms_per_step"], 4), "value": round(sm["value"], 1),
                  "unit": "TFLOP/s", "steps": K, "accum": A,
                  "gemm_tflops": round(sm["gemm_tf"], 1),

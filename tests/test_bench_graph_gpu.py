@@ -1,0 +1,79 @@
+"""Parity in the launch configuration bench.py times: the step's launches
+captured in a CUDA graph and replayed back to back (programmatic dependent
+launch lets each kernel's prologue, and the quantizer's L2 prefetch, overlap
+the kernel before it).  The replayed results must equal the eager launches bit
+for bit, the FP32 main grads must hold exactly twice one step's dW after two
+steps, and the outputs must match the oracle on sampled rows.
+
+Workload: the full hidden-2048 / FFN-6144 block at 4096 tokens (seed 4), the
+smallest configuration of the full-block sweep.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_f32_close, assert_gemm_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def step():
+    import bench
+    from fp8_block_scaled_13_b200 import build
+    build.build()
+    wl = bench.make_workload("full_block", 4096)
+    return wl, bench.Step(wl, torch.device("cuda"), n_sets=1)
+
+
+def _outputs(st):
+    return [(y.clone(), dx.clone()) for (_, _, _, y, dx) in st.out], st.grads.flat.clone()
+
+
+def test_graph_replay_matches_eager_and_oracle(step, oracle_mod):
+    wl, st = step
+    # eager: one step, weights quantized, dW added into cleared main grads
+    st.grads.zero_()
+    st.run(0, weights=True)
+    torch.cuda.synchronize()
+    assert st.fp8.device_status() == 0
+    eager, g1 = _outputs(st)
+
+    # the same two steps captured in one graph and replayed, as bench.py does
+    st.grads.zero_()
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            st.run(0, weights=True)
+            st.run(0, weights=False)
+    torch.cuda.synchronize()
+    st.grads.zero_()
+    # overwrite the outputs so that stale values cannot pass
+    for (_, _, _, y, dx) in st.out:
+        y.fill_(float("nan"))
+        dx.fill_(float("nan"))
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert st.fp8.device_status() == 0
+    replay, g2 = _outputs(st)
+    del graph
+
+    for (ye, dxe), (yr, dxr) in zip(eager, replay):
+        assert torch.equal(ye.view(torch.int16), yr.view(torch.int16))
+        assert torch.equal(dxe.view(torch.int16), dxr.view(torch.int16))
+    # two identical FP32 additions into zero: exactly twice the first
+    assert torch.equal(g2, 2.0 * g1)
+
+    # the replayed outputs against the oracle on sampled rows of every layer
+    rows = np.unique(np.linspace(0, wl.layers[0].m - 1, 12).astype(np.int64))
+    for L, (y, dx), view in zip(wl.layers, replay, st.grads.views):
+        assert_gemm_close(y[rows.tolist()], oracle_mod.linear_fprop(L.x[rows], L.w), oracle_mod,
+                          "%s fprop (graph)" % L.name)
+        assert_gemm_close(dx[rows.tolist()], oracle_mod.linear_dgrad(L.dy[rows], L.w), oracle_mod,
+                          "%s dgrad (graph)" % L.name)
+        cols = np.unique(np.linspace(0, L.n - 1, 6).astype(np.int64))
+        ref = oracle_mod.linear_wgrad(L.dy[:, cols].contiguous(), L.x)
+        assert_f32_close(view[cols.tolist()], 2.0 * ref, what="%s wgrad, two steps (graph)" % L.name)

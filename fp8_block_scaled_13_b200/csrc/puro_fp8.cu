@@ -125,7 +125,7 @@ int launch_status() {
 
 // ------------------------------------------------------------------ quant
 
-template <bool ROW, bool COL, bool BLOCK, bool RSHFL>
+template <bool ROW, bool COL, bool BLOCK, bool RSHFL, int STAGES>
 int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, const DeviceInfo& dev,
                      cudaStream_t stream) {
   int st = get_encoder();
@@ -140,8 +140,8 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, co
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return PURO_ERR_CUDA;
-  auto kern = puro::quant_kernel<ROW, COL, BLOCK, RSHFL>;
-  constexpr uint32_t smem = puro::quant_smem_bytes();
+  auto kern = puro::quant_kernel<ROW, COL, BLOCK, RSHFL, STAGES>;
+  constexpr uint32_t smem = puro::quant_smem_bytes<STAGES>();
   // per device, once (threads racing on the first call both set the same value)
   static std::atomic<bool> attr_done[kMaxDevices] = {};
   if (!attr_done[dev.index].load(std::memory_order_acquire)) {
@@ -149,7 +149,8 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, co
       return PURO_ERR_CUDA;
     attr_done[dev.index].store(true, std::memory_order_release);
   }
-  const int64_t grid = p.tiles < 2 * (int64_t)dev.sms ? p.tiles : 2 * (int64_t)dev.sms;
+  constexpr int64_t kPerSm = STAGES == 1 ? 3 : 2;  // resident CTAs per SM (shared memory)
+  const int64_t grid = p.tiles < kPerSm * dev.sms ? p.tiles : kPerSm * dev.sms;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -164,14 +165,18 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, co
   return launch_status();
 }
 
-// Row scales by shuffles when each CTA has few tiles (measured faster up to
-// about 8 tiles per CTA; the redundant per-thread form wins on long streams).
+// Short tile streams (up to about 8 tiles per CTA at two CTAs per SM): row
+// scales shared by shuffles, two stages, two CTAs per SM.  Longer streams:
+// every lane derives its rows' scales (no cross-lane latency on the encode
+// path), one stage, three CTAs per SM.  Weights (at most a few thousand
+// tiles) take two stages.  Each form was measured faster in its own range.
 template <bool ROW, bool COL, bool BLOCK>
 int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, const DeviceInfo& dev,
                  cudaStream_t stream) {
-  if (ROW && !BLOCK && p.tiles <= 8 * 2 * (int64_t)dev.sms)
-    return launch_quant_cfg<ROW, COL, BLOCK, true>(x, ld_x, p, dev, stream);
-  return launch_quant_cfg<ROW, COL, BLOCK, false>(x, ld_x, p, dev, stream);
+  const bool short_stream = p.tiles <= 8 * 2 * (int64_t)dev.sms;
+  if (BLOCK) return launch_quant_cfg<ROW, COL, BLOCK, false, 2>(x, ld_x, p, dev, stream);
+  if (short_stream) return launch_quant_cfg<ROW, COL, BLOCK, ROW, 2>(x, ld_x, p, dev, stream);
+  return launch_quant_cfg<ROW, COL, BLOCK, false, 1>(x, ld_x, p, dev, stream);
 }
 
 // ------------------------------------------------------------------ gemm

@@ -539,6 +539,8 @@ def run_ours(args):
     ceiling = None
     if rank == 0 and not args.no_ceiling:
         ceiling = fp8_ceiling(wl, dev)
+        if ceiling is not None and world == 1:
+            ceiling["sustained_same_codes"] = gemm_sustained(step, dev, smi_id(local))
 
     bf16 = None
     if not args.no_bf16:
@@ -800,6 +802,101 @@ def fp8_ceiling(wl, dev):
                 "tflops_step_shapes": round(tot_flops / (tot_ms * 1e-3) / 1e12, 1)}
     except Exception as e:  # noqa: BLE001  (library path missing on this build)
         return {"unavailable": str(e).splitlines()[0][:160]}
+
+
+def gemm_sustained(step, dev, gpu, seconds=1.0, rounds=2):
+    """Our GEMM launches against cuBLASLt's MXFP8 GEMM in the same regime: the
+    step's GEMMs alone (fprop and the fused dgrad + wgrad of every layer),
+    and the library's GEMM on the SAME E4M3 codes and shapes (fprop, dgrad,
+    wgrad per layer; the library takes 1x32 UE8M0 scales, all set to 1.0,
+    and writes BF16 where our wgrad adds FP32 into the main grads).  Each
+    side is one CUDA graph of a step's GEMMs replayed back to back for about
+    `seconds`, so both run as long, power-capped loops; the sides alternate
+    `rounds` times and the clocks are sampled over each.  None if the
+    library path is missing."""
+    import torch
+    import torch.nn.functional as F
+    if not hasattr(F, "scaled_mm") or not hasattr(torch, "float8_e8m0fnu"):
+        return None
+    fp8 = step.fp8
+    e4m3 = torch.float8_e4m3fn
+
+    def rup(a, b):
+        return (a + b - 1) // b * b
+
+    ones = {}
+
+    def unit_scales(rows, k):
+        key = (rows, k)
+        if key not in ones:
+            ones[key] = torch.full((rup(rows, 128) * rup(k // 32, 4),), 127, dtype=torch.uint8,
+                                   device=dev).view(torch.float8_e8m0fnu)
+        return ones[key]
+
+    lib_ops, flops = [], 0
+    for L, (xq, wq, dyq, _y, _dx) in zip(step.layers, step.out):
+        m, n, k = L.m, L.n, L.k
+        ops = ((xq.q, wq.q, m, n, k),                       # Y  = X W^T
+               (dyq.q, wq.qt, m, k, n),                     # dX = dY W
+               (dyq.qt[:, :m], xq.qt[:, :m], n, k, m))      # dW = dY^T X
+        for a, b, rows, cols, kk in ops:
+            lib_ops.append((a.view(e4m3), b.view(e4m3), unit_scales(rows, kk), unit_scales(cols, kk)))
+            flops += 2 * rows * cols * kk
+
+    def ours():
+        for li, (xq, wq, dyq, y, dx) in enumerate(step.out):
+            fp8.gemm_fprop(xq, wq, out=y)
+            fp8.gemm_dgrad_wgrad(dyq, wq, xq, dx=dx, dw=step.grads[li], accumulate=True)
+
+    def library():
+        for a, b, sa, sb in lib_ops:
+            F.scaled_mm(a, b.t(), sa, F.ScalingType.BlockWise1x32, sb, F.ScalingType.BlockWise1x32,
+                        swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                        output_dtype=torch.bfloat16)
+
+    try:
+        graphs = {}
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            for name, fn in (("ours", ours), ("library", library)):
+                fn()  # outside the graph first: library workspaces, attribute setup
+                torch.cuda.synchronize()
+                graphs[name] = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graphs[name], stream=cap):
+                    fn()
+        torch.cuda.synchronize()
+        res = {name: [] for name in graphs}
+        for _ in range(rounds):
+            for name, g in graphs.items():
+                g.replay()
+                t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                t0.record(); g.replay(); t1.record()
+                torch.cuda.synchronize()
+                reps = max(3, int(seconds * 1e3 / max(t0.elapsed_time(t1), 1e-3)))
+                with ClockSampler(gpu) as clk:
+                    t0.record()
+                    for _ in range(reps):
+                        g.replay()
+                    t1.record()
+                    torch.cuda.synchronize()
+                ms = t0.elapsed_time(t1) / reps
+                res[name].append({"tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+                                  "sm_mhz": clk.summary().get("sm_mhz"), "reps": reps})
+        if fp8.device_status() != 0:
+            raise RuntimeError("device status %d" % fp8.device_status())
+        del graphs
+        torch.cuda.empty_cache()
+    except Exception as e:  # noqa: BLE001  (library path missing on this build)
+        return {"unavailable": str(e).splitlines()[0][:160]}
+    mean = {name: round(statistics.mean(r["tflops"] for r in v), 1) for name, v in res.items()}
+    return {"what": "the step's GEMMs alone, ours vs cuBLASLt MXFP8 on the same E4M3 codes and "
+                    "shapes, each a graph replayed back to back for ~%.1f s, alternating %d times"
+                    % (seconds, rounds),
+            "gemm_flops_per_pass": flops,
+            "ours_tflops": mean["ours"], "library_tflops": mean["library"],
+            "ours_vs_library": round(mean["ours"] / mean["library"], 3),
+            "rounds": res}
 
 
 def run_e2e(wl, dev, K, warmup, accum):

@@ -77,3 +77,16 @@ def test_graph_replay_matches_eager_and_oracle(step, oracle_mod):
         cols = np.unique(np.linspace(0, L.n - 1, 6).astype(np.int64))
         ref = oracle_mod.linear_wgrad(L.dy[:, cols].contiguous(), L.x)
         assert_f32_close(view[cols.tolist()], 2.0 * ref, what="%s wgrad, two steps (graph)" % L.name)
+
+
+def test_sustained_library_comparison(step):
+    """The bench's like-for-like loop: our GEMM launches and the library's on
+    the same codes, both timed; our launches leave the device status clean."""
+    import bench
+    _, st = step
+    r = bench.gemm_sustained(st, torch.device("cuda"), bench.smi_id(0), seconds=0.05, rounds=1)
+    if r is None:
+        pytest.skip("torch has no MXFP8 scaled_mm on this build")
+    assert "unavailable" not in r, r
+    assert r["ours_tflops"] > 0 and r["library_tflops"] > 0
+    assert st.fp8.device_status() == 0

@@ -65,7 +65,7 @@ def load() -> ctypes.CDLL:
     P, I, INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     lib.puro_fp8_blocked_scale_bytes.argtypes = [I, I]
     lib.puro_fp8_blocked_scale_bytes.restype = I
-    lib.puro_fp8_quant_act.argtypes = [P, I, I, I, INT, P, I, P, P, I, P, P]
+    lib.puro_fp8_quant_act.argtypes = [P, I, I, I, INT, P, I, P, P, I, P, P, P]
     lib.puro_fp8_quant_weight.argtypes = [P, I, I, I, P, I, P, P, I, P, P, P]
     lib.puro_fp8_gemm_fprop.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
     lib.puro_fp8_gemm_dgrad.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
@@ -94,9 +94,10 @@ def puro_fp8_blocked_scale_bytes(rows, groups) -> int:
     return load().puro_fp8_blocked_scale_bytes(rows, groups)
 
 
-def puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, qt, ld_qt, st, stream) -> int:
+def puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, qt, ld_qt, st, tile_counter,
+                       stream) -> int:
     return load().puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, qt, ld_qt, st,
-                                     stream)
+                                     tile_counter, stream)
 
 
 def puro_fp8_quant_weight(w, n, k, ld_w, q, ld_q, s, qt, ld_qt, s_fwd, s_bwd, stream) -> int:

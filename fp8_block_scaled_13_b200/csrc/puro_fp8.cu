@@ -166,17 +166,24 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, co
 }
 
 // Short tile streams (up to about 8 tiles per CTA at two CTAs per SM): row
-// scales shared by shuffles, two stages, two CTAs per SM.  Longer streams:
-// every lane derives its rows' scales (no cross-lane latency on the encode
-// path), one stage, three CTAs per SM.  Weights (at most a few thousand
-// tiles) take two stages.  Each form was measured faster in its own range.
+// scales shared by shuffles, two stages, two CTAs per SM, a static tile
+// schedule.  Longer streams: every lane derives its rows' scales (no
+// cross-lane latency on the encode path), one stage, three CTAs per SM, and
+// the tiles after each CTA's first handed out by ticket when the caller gave
+// a tile counter (SMs stream at different rates, up to ~35% apart on a B200;
+// with a static split the launch lasts as long as its slowest SM: 32768 x
+// 12288 BOTH took 298 us static and 255 us by ticket).  Weights (at most a
+// few thousand tiles) take two stages and the static schedule.  Each form was
+// measured faster in its own range.
 template <bool ROW, bool COL, bool BLOCK>
 int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, const DeviceInfo& dev,
                  cudaStream_t stream) {
   const bool short_stream = p.tiles <= 8 * 2 * (int64_t)dev.sms;
-  if (BLOCK) return launch_quant_cfg<ROW, COL, BLOCK, false, 2>(x, ld_x, p, dev, stream);
-  if (short_stream) return launch_quant_cfg<ROW, COL, BLOCK, ROW, 2>(x, ld_x, p, dev, stream);
-  return launch_quant_cfg<ROW, COL, BLOCK, false, 1>(x, ld_x, p, dev, stream);
+  puro::QuantParams ps = p;
+  if (BLOCK || short_stream) ps.ctr = nullptr;
+  if (BLOCK) return launch_quant_cfg<ROW, COL, BLOCK, false, 2>(x, ld_x, ps, dev, stream);
+  if (short_stream) return launch_quant_cfg<ROW, COL, BLOCK, ROW, 2>(x, ld_x, ps, dev, stream);
+  return launch_quant_cfg<ROW, COL, BLOCK, false, 1>(x, ld_x, ps, dev, stream);
 }
 
 // ------------------------------------------------------------------ gemm
@@ -465,7 +472,7 @@ int64_t puro_fp8_blocked_scale_bytes(int64_t rows, int64_t groups) {
 
 int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int layout,
                        void* q, int64_t ld_q, void* s, void* qt, int64_t ld_qt, void* st,
-                       void* stream) {
+                       uint32_t* tile_counter, void* stream) {
   if (layout != PURO_ROWWISE && layout != PURO_COLWISE && layout != PURO_BOTH)
     return PURO_ERR_LAYOUT;
   if (rows < 0 || cols < 0 || rows >= kMaxDim || cols >= kMaxDim) return PURO_ERR_SHAPE;
@@ -485,9 +492,11 @@ int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x, 
     if (!st) return PURO_ERR_NULL;
     if (!aligned16(st)) return PURO_ERR_ALIGN;
   }
+  if (reinterpret_cast<uintptr_t>(tile_counter) % 8) return PURO_ERR_ALIGN;
   DeviceInfo* dev = nullptr;
   if ((r = current_device(&dev)) != PURO_OK) return r;
   puro::QuantParams p{};
+  p.ctr = tile_counter;
   p.rows = rows;
   p.cols = cols;
   p.q = static_cast<uint8_t*>(q);

@@ -70,6 +70,11 @@ struct QuantParams {
   uint8_t* sw_bwd;  // BLOCK: optional blocked, cols x rows/128 groups
   int64_t bwd_g4;
   int32_t tiles_c, tiles;
+  // Optional tile counter pair (two zeroed 32-bit words; null: static
+  // schedule).  Each CTA takes its first STAGES tiles statically and the rest
+  // by ticket, so SMs that stream faster take more tiles; the last CTA to
+  // finish sets both words back to zero.
+  uint32_t* ctr;
 };
 
 // Scale exponents of two groups at once.  a2 holds two amax magnitudes (BF16
@@ -274,14 +279,16 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
   float* col_scale = reinterpret_cast<float*>(col_part + kWarps * 64);  // [128] 2^-e per column
   uint32_t* blk_part = reinterpret_cast<uint32_t*>(col_scale + 128);    // [8]
   uint64_t* full = reinterpret_cast<uint64_t*>(blk_part + kWarps);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + STAGES);
+  int2* tile_rc = reinterpret_cast<int2*>(full + STAGES);  // [STAGES] (row, col) tile of the stage
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tile_rc + STAGES);
 
   const int tid = threadIdx.x;
   const int i = tid >> 4, j = tid & 15, warp = tid >> 5;
-  // tiles t = blockIdx.x + it * gridDim.x, walked as (row tile, col tile)
-  const int32_t tc_step = (int32_t)(gridDim.x % p.tiles_c), tr_step = (int32_t)(gridDim.x / p.tiles_c);
-  const int32_t my_tiles =
-      (int32_t)blockIdx.x < p.tiles ? (p.tiles - (int32_t)blockIdx.x + (int32_t)gridDim.x - 1) / (int32_t)gridDim.x : 0;
+  // Tile t is (row tile t / tiles_c, col tile t % tiles_c).  Load k of this
+  // CTA fetches tile blockIdx.x + k * gridDim.x; with a tile counter, loads
+  // from STAGES on fetch tile STAGES * gridDim.x + ticket instead.  The tile
+  // of each load is published in tile_rc (-1: no more tiles).
+  const bool dyn = p.ctr != nullptr;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
@@ -295,53 +302,67 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
     // still finishing.  A prefetch only moves data into L2, the point of
     // coherence, and the loads that fill shared memory still follow the
     // dependency wait below, so a producer's later writes are what they read.
-    int32_t r = (int32_t)blockIdx.x / p.tiles_c, c = (int32_t)blockIdx.x % p.tiles_c;
-    for (int32_t t = 0; t < STAGES && t < my_tiles; ++t) {
-      tma_prefetch_l2_2d(&tm_x, c * 128, r * 128);
-      c += tc_step;
-      r += tr_step;
-      if (c >= p.tiles_c) { c -= p.tiles_c; ++r; }
+    for (int32_t k = 0; k < STAGES; ++k) {
+      const int32_t t = (int32_t)blockIdx.x + k * (int32_t)gridDim.x;
+      if (t >= p.tiles) break;
+      const int32_t r = t / p.tiles_c;
+      tma_prefetch_l2_2d(&tm_x, (t - r * p.tiles_c) * 128, r * 128);
     }
   }
   // the input may come from the kernel just before this one on the stream
   pdl_wait();
   pdl_trigger();
-  // producer-side tile cursor (thread 0 only)
-  int32_t ptr_r = (int32_t)blockIdx.x / p.tiles_c, ptr_c = (int32_t)blockIdx.x % p.tiles_c;
+  // producer state (thread 0 only): loads issued, whether the end marker
+  // went out, and the ticket for the next load (taken one load ahead, so its
+  // round trip overlaps a tile of work)
   int32_t p_it = 0;
+  bool p_end = false;
+  uint32_t ticket = 0;
   auto issue_next = [&]() {
+    if (p_end) return;
     const int s = p_it % STAGES;
-    mbar_arrive_expect_tx(&full[s], kQTileBytes);
-    tma_load_2d<1>(tiles + s * kQTileBytes, &tm_x, ptr_c * 128, ptr_r * 128, smem_u32(&full[s]));
+    const int32_t t = (dyn && p_it >= STAGES) ? STAGES * (int32_t)gridDim.x + (int32_t)ticket
+                                               : (int32_t)blockIdx.x + p_it * (int32_t)gridDim.x;
     ++p_it;
-    ptr_c += tc_step;
-    ptr_r += tr_step;
-    if (ptr_c >= p.tiles_c) { ptr_c -= p.tiles_c; ++ptr_r; }
+    if (t < p.tiles) {
+      const int32_t r = t / p.tiles_c, c = t - r * p.tiles_c;
+      tile_rc[s] = make_int2(r, c);
+      mbar_arrive_expect_tx(&full[s], kQTileBytes);
+      tma_load_2d<1>(tiles + s * kQTileBytes, &tm_x, c * 128, r * 128, smem_u32(&full[s]));
+      if (dyn && p_it >= STAGES) ticket = atomicAdd(p.ctr, 1u);
+    } else {
+      tile_rc[s] = make_int2(-1, -1);
+      mbar_arrive(&full[s]);
+      p_end = true;
+    }
   };
   if (tid == 0)
-    while (p_it < my_tiles && p_it < STAGES) issue_next();
+    for (int k = 0; k < STAGES; ++k) issue_next();
 
   // per-thread constants of the output addressing
   const uint32_t s_own_row = blocked_in_chunk(8 * i + (j & 7));    // row scale byte (j < 8)
   const uint32_t s_half_chunk = blocked_in_chunk(8 * i + (j >> 1));  // the same, row j >> 1
   const uint32_t st_in_chunk = blocked_in_chunk(2 * (tid & 63));     // column scale bytes (tid < 64)
 
-  int32_t tr = (int32_t)blockIdx.x / p.tiles_c, tc = (int32_t)blockIdx.x % p.tiles_c;
   int32_t prev_r0 = 0, prev_c0 = 0;  // the tile whose transposed codes wait in qt_buf
-  for (int32_t it = 0; it < my_tiles; ++it) {
-    const int32_t r0 = tr * 128, c0 = tc * 128;
+  int32_t it = 0;
+  for (;; ++it) {
     const int s = it % STAGES;
     const bool ok = mbar_wait(&full[s], (uint32_t)((it / STAGES) & 1), abort_flag);
+    const int2 rc = ok ? tile_rc[s] : make_int2(-1, -1);
+    const int32_t tr = rc.x, tc = rc.y;
+    const int32_t r0 = tr * 128, c0 = tc * 128;
     // this thread's 8 rows x 8 columns; rows past the end were filled with 0
     uint4 v[8];
     const uint8_t* tile = tiles + s * kQTileBytes + (8 * i) * 256 + 16 * j;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = ok ? lds_v4(tile + k * 256) : make_uint4(0, 0, 0, 0);
+    for (int k = 0; k < 8; ++k) v[k] = (ok && tr >= 0) ? lds_v4(tile + k * 256) : make_uint4(0, 0, 0, 0);
     // every thread holds its part: stage s is free again, and every thread
     // has finished the previous tile, its transposed codes included (and if
-    // any wait gave up, the whole block stops here together)
-    if (__syncthreads_or(!ok)) break;
-    if (tid == 0 && p_it < my_tiles) issue_next();
+    // any wait gave up, the whole block stops here together; every thread
+    // read the same end marker)
+    if (__syncthreads_or(!ok) || tr < 0) break;
+    if (tid == 0) issue_next();
     if (COL && it > 0) qt_readout(p, qt_buf + ((it - 1) & 1) * kQtTileBytes, prev_r0, prev_c0, tid);
 
     // ---- magnitudes: per-row amax of this thread's 8 columns (two rows per
@@ -531,14 +552,20 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
     // other transposed buffer) are next written after the barrier at the top
     // of the next iteration, which no thread passes before every thread has
     // finished this tile.
-    tc += tc_step;
-    tr += tr_step;
-    if (tc >= p.tiles_c) { tc -= p.tiles_c; ++tr; }
   }
   // the last tile's transposed codes (if every wait succeeded)
-  if (COL && my_tiles > 0) {
+  if (COL && it > 0) {
     if (!__syncthreads_or(*abort_flag != 0))
-      qt_readout(p, qt_buf + ((my_tiles - 1) & 1) * kQtTileBytes, prev_r0, prev_c0, tid);
+      qt_readout(p, qt_buf + ((it - 1) & 1) * kQtTileBytes, prev_r0, prev_c0, tid);
+  }
+  // the last CTA out resets the tile counter for the next launch (every
+  // ticket of every CTA was taken before its arrival here)
+  if (dyn && tid == 0) {
+    __threadfence();
+    if (atomicAdd(p.ctr + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.ctr, 0u);
+      atomicExch(p.ctr + 1, 0u);
+    }
   }
   // Copies are only issued for tiles this CTA processes, and each one was
   // waited for above, unless a wait gave up; then let the outstanding ones
@@ -556,7 +583,7 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
 template <int STAGES>
 constexpr uint32_t quant_smem_bytes() {
   return STAGES * kQTileBytes + 2 * kQtTileBytes + (kQThreads / 32) * 64 * 4 + 128 * 4 +
-         (kQThreads / 32) * 4 + STAGES * 8 + 16 + 1024;
+         (kQThreads / 32) * 4 + STAGES * 8 + STAGES * 8 + 16 + 1024;
 }
 
 }  // namespace puro

@@ -147,6 +147,11 @@ class QuantAct:
     s: torch.Tensor | None = None    # blocked: rows x cols/128 groups
     qt: torch.Tensor | None = None   # [cols, ld_qt] u8, transposed codes
     st: torch.Tensor | None = None   # blocked: cols x ceil(rows/128) groups
+    # two int32 words, zero before first use, that the quantizer may hand its
+    # tiles out from (None: static tile schedule); every call leaves them
+    # zero.  Calls that may run at the same time need distinct outputs, and so
+    # distinct words.
+    work: torch.Tensor | None = None
 
 
 @dataclass
@@ -175,6 +180,7 @@ def quant_act(x: torch.Tensor, layout: str = "both", out: QuantAct | None = None
         if flag & _lib.PURO_COLWISE:
             out.qt = torch.empty((cols, _round16(rows)), dtype=torch.uint8, device=dev)
             out.st = _blocked(cols, (rows + 127) // 128, dev)
+        out.work = torch.zeros(2, dtype=torch.int32, device=dev)
     else:
         if (out.rows, out.cols) != (rows, cols):
             raise ValueError("out was made for a [%d, %d] input" % (out.rows, out.cols))
@@ -187,12 +193,15 @@ def quant_act(x: torch.Tensor, layout: str = "both", out: QuantAct | None = None
                           (torch.uint8,), "out.qt", min_cols=True)
             _check_bytes(_need(out.st, "out has no transposed scales"),
                          blocked_scale_bytes(cols, (rows + 127) // 128), "out.st")
+        if out.work is not None and (not out.work.is_cuda or out.work.dtype != torch.int32
+                                     or not out.work.is_contiguous() or out.work.numel() < 2):
+            raise ValueError("out.work must be a contiguous CUDA int32 tensor of at least 2 elements")
     ptr = lambda t: t.data_ptr() if t is not None else None
     st = _lib.puro_fp8_quant_act(
         x.data_ptr(), rows, cols, x.stride(0), flag,
         ptr(out.q), out.q.stride(0) if out.q is not None else 0, ptr(out.s),
         ptr(out.qt), out.qt.stride(0) if out.qt is not None else 0, ptr(out.st),
-        _stream())
+        ptr(out.work), _stream())
     _check(st, "puro_fp8_quant_act")
     return out
 

@@ -110,11 +110,23 @@ PURO_API int64_t puro_fp8_blocked_scale_bytes(int64_t rows, int64_t groups);
  *        x[128g .. min(128g+127, rows-1), c] -- the last group may be short
  *        and only its valid rows enter the amax.
  * Unused outputs may be NULL.  rows == 0 or cols == 0 is a no-op.
+ *
+ * tile_counter : NULL, or two 32-bit words of device memory, 8-byte aligned,
+ *   owned by the caller and zero before the first call that gets them.  On
+ *   long inputs (more than about 16 tiles of 128 x 128 per SM) the call then
+ *   hands the tiles out by ticket from this counter, which keeps every SM
+ *   busy to the end; NULL, or a shorter input, takes a static tile schedule.
+ *   The results are the same either way.  Every call leaves the words zero
+ *   when its kernel completes, so one counter serves any number of calls in
+ *   stream order (CUDA graph replays included).  Calls that may run at the
+ *   same time on the GPU need distinct counters -- one per output set is
+ *   natural, since such calls need distinct outputs anyway.
  * Limits: rows, cols < 2^31.
  */
 PURO_API int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
                                 int layout, void* q, int64_t ld_q, void* s,
-                                void* qt, int64_t ld_qt, void* st, void* stream);
+                                void* qt, int64_t ld_qt, void* st, uint32_t* tile_counter,
+                                void* stream);
 
 /*
  * puro_fp8_quant_weight -- 128x128 block quantization of a weight: one

@@ -54,7 +54,7 @@ A = 1 << 20  # a 16-byte-aligned fake device address; never dereferenced here
 
 
 @pytest.mark.parametrize("args,code", [
-    # (x, rows, cols, ld_x, layout, q, ld_q, s, qt, ld_qt, st)
+    # (x, rows, cols, ld_x, layout, q, ld_q, s, qt, ld_qt, st[, tile_counter])
     ((A, 16, 128, 128, 7, A, 128, A, None, 0, None), -4),     # bad layout flag
     ((A, 16, 100, 128, 1, A, 128, A, None, 0, None), -3),     # cols not a multiple of 128
     ((A, -1, 128, 128, 1, A, 128, A, None, 0, None), -3),     # negative rows
@@ -67,14 +67,16 @@ A = 1 << 20  # a 16-byte-aligned fake device address; never dereferenced here
     ((A, 16, 128, 128, 1, A, 128, A + 8, None, 0, None), -2), # misaligned s
     ((A, 17, 128, 128, 2, None, 0, None, A, 16, A), -3),      # qt leading dim below rows rounded to 16
     ((A, 16, 128, 128, 2, None, 0, None, A, 16, None), -1),   # COLWISE without st
+    ((A, 16, 128, 128, 1, A, 128, A, None, 0, None, A + 4), -2),  # tile counter not 8-byte aligned
 ])
 def test_quant_act_argument_errors(lib, args, code):
+    args = args + (None,) * (12 - len(args))
     assert lib.puro_fp8_quant_act(*args, None) == code
 
 
 def test_quant_act_empty_is_noop(lib):
-    assert lib.puro_fp8_quant_act(None, 0, 128, 128, 3, None, 0, None, None, 0, None, None) == 0
-    assert lib.puro_fp8_quant_act(None, 5, 0, 0, 3, None, 0, None, None, 0, None, None) == 0
+    assert lib.puro_fp8_quant_act(None, 0, 128, 128, 3, None, 0, None, None, 0, None, None, None) == 0
+    assert lib.puro_fp8_quant_act(None, 5, 0, 0, 3, None, 0, None, None, 0, None, None, None) == 0
 
 
 @pytest.mark.parametrize("args,code", [

@@ -181,3 +181,82 @@ def test_blocked_layout_padding_rows(fp8):
 def test_blocked_index_is_a_bijection():
     idx = blocked_index(384, 8)
     assert np.unique(idx).size == idx.size and idx.max() == 3 * 2 * 512 - 1
+
+
+def _outs(xq):
+    """Every byte the call defines: the codes (the transposed codes with their
+    zero padding columns) and the scale bytes of the existing groups (the
+    padding groups of a blocked array are not written)."""
+    torch.cuda.synchronize()
+    out = []
+    if xq.q is not None:
+        q, s = gpu_rowwise(xq)
+        out += [q.copy(), s.copy()]
+    if xq.qt is not None:
+        out += [np_u8(xq.qt).copy(), gpu_colwise(xq)[1].copy()]
+    return out
+
+
+def _same(a, b):
+    return len(a) == len(b) and all(np.array_equal(x, y) for x, y in zip(a, b))
+
+
+def _long_stream(rows, cols):
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return -(-rows // 128) * (cols // 128) > 16 * sms
+
+
+@pytest.mark.parametrize("rows,cols,layout", [(40000, 1024, "both"), (33001, 2048, "rowwise"),
+                                              (20000, 2048, "colwise")])
+def test_tile_counter_long_streams(fp8, oracle_mod, rows, cols, layout):
+    """Long inputs (more than 16 tiles per SM) hand their tiles out by ticket
+    from the output's counter: the oracle's bytes over the whole tensor (ragged
+    last row tile included), the same bytes as the static schedule, and the
+    counter back at zero after every call."""
+    assert _long_stream(rows, cols)
+    x = _rand((rows, cols), rows + cols)
+    xq = _check_all(fp8, oracle_mod, x, layout)
+    assert xq.work is not None and not xq.work.any(), "tile counter not reset"
+    ref = _outs(xq)
+    xc = x.cuda()
+    for _ in range(2):  # the same counter again: same bytes
+        fp8.quant_act(xc, layout, out=xq)
+        torch.cuda.synchronize()
+        assert not xq.work.any(), "tile counter not reset"
+        assert _same(ref, _outs(xq))
+    static = fp8.quant_act(xc, layout)
+    static.work = None
+    for t in (static.q, static.s, static.qt, static.st):
+        if t is not None:
+            t.zero_()
+    fp8.quant_act(xc, layout, out=static)
+    torch.cuda.synchronize()
+    assert fp8.device_status() == 0
+    assert _same(ref, _outs(static))
+
+
+def test_tile_counter_graph_replays(fp8):
+    """Two ticket-scheduled launches captured in one CUDA graph on the same
+    counter, replayed three times: every replay rewrites the same bytes and
+    leaves the counter at zero."""
+    x = _rand((40000, 1024), 9).cuda()
+    xq = fp8.quant_act(x, "both")
+    torch.cuda.synchronize()
+    ref = _outs(xq)
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            fp8.quant_act(x, "both", out=xq)
+            fp8.quant_act(x, "both", out=xq)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for t in (xq.q, xq.s, xq.qt, xq.st):
+            t.fill_(0x5A)
+        g.replay()
+        torch.cuda.synchronize()
+        assert fp8.device_status() == 0
+        assert not xq.work.any(), "tile counter not reset"
+        assert _same(ref, _outs(xq))
+    del g

@@ -31,6 +31,7 @@ PURO_DW_F32_ACCUMULATE = 2
 EXPORTS = (
     "puro_fp8_blocked_scale_bytes",
     "puro_fp8_quant_act",
+    "puro_fp8_quant_act_static_scratch",
     "puro_fp8_quant_weight",
     "puro_fp8_gemm_fprop",
     "puro_fp8_gemm_dgrad",
@@ -66,6 +67,7 @@ def load() -> ctypes.CDLL:
     lib.puro_fp8_blocked_scale_bytes.argtypes = [I, I]
     lib.puro_fp8_blocked_scale_bytes.restype = I
     lib.puro_fp8_quant_act.argtypes = [P, I, I, I, INT, P, I, P, P, I, P, P, P]
+    lib.puro_fp8_quant_act_static_scratch.argtypes = [P, I, I, I, INT, P, I, P, P, I, P, P]
     lib.puro_fp8_quant_weight.argtypes = [P, I, I, I, P, I, P, P, I, P, P, P]
     lib.puro_fp8_gemm_fprop.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]
     lib.puro_fp8_gemm_dgrad.argtypes = [P, I, P, P, I, P, P, I, I, I, I, P]

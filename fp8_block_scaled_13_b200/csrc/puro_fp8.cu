@@ -677,3 +677,56 @@ extern "C" int puro_fp8_test_bounded_wait(int64_t limit_ns, void* stream) {
       (uint64_t)limit_ns);
   return launch_status();
 }
+
+// ---------------------------------------------------------------- static-scratch entry point
+//
+// Some callers cannot hand this library any device memory beyond their inputs
+// and outputs: an engine that reserves the GPU's memory for its own pool at
+// start-up leaves nothing for cudaMalloc (which then fails, or stalls the
+// device while the pool gives memory back), and a C caller that only holds
+// the buffers it was given has no allocator to ask.  For them, the
+// quantizer's tile counter lives in this file-scope array instead: 256
+// bytes (one counter pair is used) in the library's own device memory, held
+// by every GPU that loads the library until the process exits.  Host code
+// needs its device address, which cudaGetSymbolAddress gives once per device
+// (the symbol's name is only a host-side stand-in).
+namespace {
+
+constexpr size_t kStaticScratchBytes = 256;
+static __device__ __align__(256) uint32_t g_static_scratch[kStaticScratchBytes / 4];
+uint32_t* g_static_scratch_addr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" int puro_fp8_quant_act_static_scratch(const void* x, int64_t rows, int64_t cols,
+                                                 int64_t ld_x, int layout, void* q, int64_t ld_q,
+                                                 void* s, void* qt, int64_t ld_qt, void* st,
+                                                 void* stream) {
+  // the sizes this entry point takes (the rest is checked by the common path)
+  if (layout != PURO_ROWWISE && layout != PURO_COLWISE && layout != PURO_BOTH)
+    return PURO_ERR_LAYOUT;
+  if (rows < 0 || cols < 0 || rows >= kMaxDim || cols >= kMaxDim || cols % 128) return PURO_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return PURO_OK;
+  // the counter's 32-bit tickets: at most one per tile plus one per CTA
+  if ((cols / 128) * ((rows + 127) / 128) >= kMaxDim) return PURO_ERR_SHAPE;
+  DeviceInfo* dev = nullptr;
+  int r = current_device(&dev);
+  if (r != PURO_OK) return r;
+  uint32_t* ctr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_static_scratch_addr[dev->index]) {
+      void* a = nullptr;
+      if (cudaGetSymbolAddress(&a, g_static_scratch) != cudaSuccess || a == nullptr)
+        return PURO_ERR_CUDA;
+      g_static_scratch_addr[dev->index] = static_cast<uint32_t*>(a);
+    }
+    ctr = g_static_scratch_addr[dev->index];
+  }
+  // The counter must start at zero.  Each call clears it on its stream before
+  // its kernel (the kernel also leaves it zero), so a call that ended early
+  // leaves nothing behind; calls that overlap on the GPU share it and race.
+  if (cudaMemsetAsync(ctr, 0, 2 * sizeof(uint32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PURO_ERR_CUDA;
+  return puro_fp8_quant_act(x, rows, cols, ld_x, layout, q, ld_q, s, qt, ld_qt, st, ctr, stream);
+}

@@ -129,6 +129,38 @@ PURO_API int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64
                                 void* stream);
 
 /*
+ * puro_fp8_quant_act_static_scratch -- puro_fp8_quant_act for callers that
+ * cannot provide the tile counter's eight bytes of device memory.  (A support
+ * call of this library; the paper has no counterpart.)
+ *
+ * Who needs it: a caller that owns no device memory besides its inputs and
+ * outputs -- an engine that hands the GPU's memory to its own pool at
+ * start-up, so that a cudaMalloc would fail or stall the device, or a C
+ * caller that was only given the buffers it works on.  Passing a NULL
+ * tile_counter to puro_fp8_quant_act also allocates nothing, but then long
+ * inputs run on the static tile schedule, which waits for the slowest SM.
+ *
+ * Arguments, layouts, results and errors are those of puro_fp8_quant_act.
+ * The counter lives in a 256-byte array in this library's device memory
+ * (one counter pair is used; every GPU that loads the library holds the
+ * array until the process exits).  Nothing is allocated: no cudaMalloc,
+ * cudaFree or allocating library call.
+ * - The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - Every call clears the counter on `stream` before its kernel.  All calls
+ *   share the one array, so calls whose kernels may overlap on the GPU
+ *   (other streams) race on it and must not be made; stream-ordered calls are
+ *   safe.
+ * - Limit: fewer than 2^31 tiles of 128 x 128 (the counter hands out 32-bit
+ *   tickets), as for puro_fp8_quant_act; larger inputs return PURO_ERR_SHAPE.
+ */
+PURO_API int puro_fp8_quant_act_static_scratch(const void* x, int64_t rows, int64_t cols,
+                                               int64_t ld_x, int layout, void* q, int64_t ld_q,
+                                               void* s, void* qt, int64_t ld_qt, void* st,
+                                               void* stream);
+
+/*
  * puro_fp8_quant_weight -- 128x128 block quantization of a weight: one
  * power-of-two scale, computed online, for each 128x128 block
  * (paper.rainbus.top summary, background "FP8 块级混合精度训练" and

@@ -198,3 +198,17 @@ def test_oracle_never_imports_product():
             src = open(os.path.join(odir, f)).read()
             includes = re.findall(r'#include\s*[<"]([^>"]+)', src)
             assert not any("puro_fp8" in h or h.startswith("cuda") for h in includes), includes
+
+
+def test_static_scratch_entry_rejects_before_cuda(lib):
+    """The allocation-free quantizer entry point checks its sizes before it
+    touches the device: a bad layout, a bad shape, and an input of 2^31 or
+    more tiles (the tile counter's limit) come back as errors, and an empty
+    input is a no-op."""
+    f = lib.load().puro_fp8_quant_act_static_scratch
+    args = lambda rows, cols, layout: (A, rows, cols, cols, layout, A, cols, A, A, 16, A, None)
+    assert f(*args(16, 128, 7)) == -4
+    assert f(*args(16, 100, 3)) == -3
+    assert f(*args(-1, 128, 3)) == -3
+    assert f(*args(32768, (1 << 31) - 128, 3)) == -3
+    assert f(*args(0, 128, 3)) == 0

@@ -70,10 +70,13 @@ struct QuantParams {
   uint8_t* sw_bwd;  // BLOCK: optional blocked, cols x rows/128 groups
   int64_t bwd_g4;
   int32_t tiles_c, tiles;
-  // Optional tile counter pair (two zeroed 32-bit words; null: static
-  // schedule).  Each CTA takes its first STAGES tiles statically and the rest
-  // by ticket, so SMs that stream faster take more tiles; the last CTA to
-  // finish sets both words back to zero.
+  // Optional tile counter (a zeroed 32-bit word; null: static schedule),
+  // used with one stage only.  Each CTA takes its first tile statically and
+  // the rest by ticket, so SMs that stream faster take more tiles.  Tickets
+  // 0 .. tiles-1 go out in order (the valid ones map to tiles gridDim.x ..
+  // tiles-1, and each CTA stops at its first invalid one), so the CTA that
+  // draws ticket tiles-1 knows every other CTA has drawn its last, and sets
+  // the counter back to zero.
   uint32_t* ctr;
 };
 
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
   // CTA fetches tile blockIdx.x + k * gridDim.x; with a tile counter, loads
   // from STAGES on fetch tile STAGES * gridDim.x + ticket instead.  The tile
   // of each load is published in tile_rc (-1: no more tiles).
-  const bool dyn = p.ctr != nullptr;
+  const bool dyn = STAGES == 1 && p.ctr != nullptr;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
@@ -321,8 +324,10 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
   auto issue_next = [&]() {
     if (p_end) return;
     const int s = p_it % STAGES;
-    const int32_t t = (dyn && p_it >= STAGES) ? STAGES * (int32_t)gridDim.x + (int32_t)ticket
-                                               : (int32_t)blockIdx.x + p_it * (int32_t)gridDim.x;
+    const bool by_ticket = dyn && p_it >= STAGES;
+    const int32_t t = by_ticket ? STAGES * (int32_t)gridDim.x + (int32_t)ticket
+                                : (int32_t)blockIdx.x + p_it * (int32_t)gridDim.x;
+    if (by_ticket && ticket == (uint32_t)(p.tiles - 1)) atomicExch(p.ctr, 0u);
     ++p_it;
     if (t < p.tiles) {
       const int32_t r = t / p.tiles_c, c = t - r * p.tiles_c;
@@ -557,15 +562,6 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
   if (COL && it > 0) {
     if (!__syncthreads_or(*abort_flag != 0))
       qt_readout(p, qt_buf + ((it - 1) & 1) * kQtTileBytes, prev_r0, prev_c0, tid);
-  }
-  // the last CTA out resets the tile counter for the next launch (every
-  // ticket of every CTA was taken before its arrival here)
-  if (dyn && tid == 0) {
-    __threadfence();
-    if (atomicAdd(p.ctr + 1, 1u) == gridDim.x - 1) {
-      atomicExch(p.ctr, 0u);
-      atomicExch(p.ctr + 1, 0u);
-    }
   }
   // Copies are only issued for tiles this CTA processes, and each one was
   // waited for above, unless a wait gave up; then let the outstanding ones

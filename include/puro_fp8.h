@@ -116,11 +116,13 @@ PURO_API int64_t puro_fp8_blocked_scale_bytes(int64_t rows, int64_t groups);
  *   long inputs (more than about 16 tiles of 128 x 128 per SM) the call then
  *   hands the tiles out by ticket from this counter, which keeps every SM
  *   busy to the end; NULL, or a shorter input, takes a static tile schedule.
- *   The results are the same either way.  Every call leaves the words zero
- *   when its kernel completes, so one counter serves any number of calls in
- *   stream order (CUDA graph replays included).  Calls that may run at the
- *   same time on the GPU need distinct counters -- one per output set is
- *   natural, since such calls need distinct outputs anyway.
+ *   The results are the same either way.  Every call that completes leaves
+ *   the words zero (the CTA that draws the last ticket clears the counter), so
+ *   one counter serves any number of calls in stream order (CUDA graph
+ *   replays included); after a call that reported PURO_ERR_DEVICE_TIMEOUT,
+ *   clear it before using it again.  Calls that may run at the same time on
+ *   the GPU need distinct counters -- one per output set is natural, since
+ *   such calls need distinct outputs anyway.
  * Limits: rows, cols < 2^31.
  */
 PURO_API int puro_fp8_quant_act(const void* x, int64_t rows, int64_t cols, int64_t ld_x,

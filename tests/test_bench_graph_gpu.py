@@ -5,8 +5,10 @@ the kernel before it).  The replayed results must equal the eager launches bit
 for bit, the FP32 main grads must hold exactly twice one step's dW after two
 steps, and the outputs must match the oracle on sampled rows.
 
-Workload: the full hidden-2048 / FFN-6144 block at 4096 tokens (seed 4), the
-smallest configuration of the full-block sweep.
+Workloads: the full hidden-2048 / FFN-6144 block (seed 4) at 4096 tokens, the
+smallest configuration of the full-block sweep (every quantizer launch a short
+stream with a static tile schedule), and at 32768 tokens, the default bench
+line (the activation quantizers hand their tiles out by ticket).
 """
 import numpy as np
 import pytest
@@ -17,13 +19,16 @@ from helpers import assert_f32_close, assert_gemm_close
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def step():
+@pytest.fixture(scope="module", params=[4096, 32768])
+def step(request):
     import bench
     from fp8_block_scaled_13_b200 import build
     build.build()
-    wl = bench.make_workload("full_block", 4096)
-    return wl, bench.Step(wl, torch.device("cuda"), n_sets=1)
+    wl = bench.make_workload("full_block", request.param)
+    st = bench.Step(wl, torch.device("cuda"), n_sets=1)
+    yield wl, st
+    del st
+    torch.cuda.empty_cache()
 
 
 def _outputs(st):

@@ -165,25 +165,35 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, co
   return launch_status();
 }
 
-// Short tile streams (up to about 8 tiles per CTA at two CTAs per SM): row
-// scales shared by shuffles, two stages, two CTAs per SM, a static tile
-// schedule.  Longer streams: every lane derives its rows' scales (no
-// cross-lane latency on the encode path), one stage, three CTAs per SM, and
-// the tiles after each CTA's first handed out by ticket when the caller gave
-// a tile counter (SMs stream at different rates, up to ~35% apart on a B200;
-// with a static split the launch lasts as long as its slowest SM: 32768 x
-// 12288 BOTH took 298 us static and 255 us by ticket).  Weights (at most a
-// few thousand tiles) take two stages and the static schedule.  Each form was
-// measured faster in its own range.
+// Short tile streams (up to about 8 tiles per CTA at two CTAs per SM): two
+// stages, two CTAs per SM, a static tile schedule.  Longer streams: one
+// stage, three CTAs per SM, and the tiles after each CTA's first handed out
+// by ticket when the caller gave a tile counter (SMs stream at different
+// rates, up to ~35% apart on a B200; with a static split the launch lasts as
+// long as its slowest SM: 32768 x 12288 BOTH took 298 us static and 255 us by
+// ticket).  Activations share their row scales by shuffles in both forms
+// (7% fewer instructions than every lane deriving its own; with three CTAs
+// per SM there are warps enough to hide the shuffles' latency).  Weights (at
+// most a few thousand tiles) take two stages and the static schedule.  Each
+// form was measured faster in its own range.
 template <bool ROW, bool COL, bool BLOCK>
 int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, const DeviceInfo& dev,
                  cudaStream_t stream) {
   const bool short_stream = p.tiles <= 8 * 2 * (int64_t)dev.sms;
   puro::QuantParams ps = p;
   if (BLOCK || short_stream) ps.ctr = nullptr;
+  // the kernel's division-free tile decode (tiles_c >= 1 here; < 2^24)
+  ps.tc_magic = 0;
+  ps.tc_shift = 0;
+  if (ps.tiles_c > 1) {
+    int l = 0;
+    while ((int64_t(1) << l) < ps.tiles_c) ++l;
+    ps.tc_magic = (uint32_t)(((uint64_t(1) << (31 + l)) + (uint64_t)ps.tiles_c - 1) / (uint64_t)ps.tiles_c);
+    ps.tc_shift = l - 1;
+  }
   if (BLOCK) return launch_quant_cfg<ROW, COL, BLOCK, false, 2>(x, ld_x, ps, dev, stream);
   if (short_stream) return launch_quant_cfg<ROW, COL, BLOCK, ROW, 2>(x, ld_x, ps, dev, stream);
-  return launch_quant_cfg<ROW, COL, BLOCK, false, 1>(x, ld_x, ps, dev, stream);
+  return launch_quant_cfg<ROW, COL, BLOCK, ROW, 1>(x, ld_x, ps, dev, stream);
 }
 
 // ------------------------------------------------------------------ gemm

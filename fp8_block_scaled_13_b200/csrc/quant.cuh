@@ -8,17 +8,18 @@
 // e clamped to [-127, 127], and every element is encoded round-to-nearest-even
 // with saturation.
 //
-// One persistent kernel serves every layout.  Each CTA (256 threads, two per
-// SM, so two tiles are processed side by side) walks a strided list of
+// One persistent kernel serves every layout.  Each CTA (256 threads; two or
+// three per SM, so as many tiles are processed side by side) walks a list of
 // 128x128 tiles of the BF16 input; a TMA ring of STAGES 32 KB tile buffers
 // keeps the next tiles in flight while the current one is processed, and a
 // stage is handed back to the TMA as soon as every thread has copied its part
 // into registers.  Long tile streams run one stage and three CTAs per SM (the
 // next tile's load still has a whole tile's processing time to land, and the
-// third CTA hides more latency: 2-3% faster on 4096+ tiles); short streams keep
-// two stages and two CTAs per SM (the first tiles are also prefetched into L2 before the
-// kernel waits on its predecessor).  Thread (i, j) = (tid/16, tid%16) holds
-// rows 8i..8i+7 and columns 8j..8j+7.  From those registers:
+// third CTA hides more latency: 2-3% faster on 4096+ tiles), the tiles after
+// each CTA's first handed out by ticket; short streams keep two stages, two
+// CTAs per SM and a static list (the first tiles are also prefetched into L2
+// before the kernel waits on its predecessor).  Thread (i, j) = (tid/16,
+// tid%16) holds rows 8i..8i+7 and columns 8j..8j+7.  From those registers:
 //   ROW   : row amax by a 16-lane shuffle reduction; codes stored in place.
 //   COL   : column amax by a shuffle + shared-memory reduction over the 8
 //           warps; codes transposed through an XOR-swizzled 16 KB shared tile
@@ -70,6 +71,15 @@ struct QuantParams {
   uint8_t* sw_bwd;  // BLOCK: optional blocked, cols x rows/128 groups
   int64_t bwd_g4;
   int32_t tiles_c, tiles;
+  // Row tile of tile t without a division: t / tiles_c == umulhi(t,
+  // tc_magic) >> tc_shift for every t < 2^31 when tiles_c > 1 (set by the
+  // launcher: l = ceil(log2(tiles_c)), tc_magic = ceil(2^(31+l) / tiles_c),
+  // tc_shift = l - 1; the product's error stays below 1 / tiles_c).  The
+  // producer thread decodes every tile it loads, and the rest of the block
+  // waits for it at the stage barrier: a 32-bit division there cost ~2 us per
+  // 4096-tile launch.
+  uint32_t tc_magic;
+  int32_t tc_shift;
   // Optional tile counter (a zeroed 32-bit word; null: static schedule),
   // used with one stage only.  Each CTA takes its first tile statically and
   // the rest by ticket, so SMs that stream faster take more tiles.  Tickets
@@ -230,6 +240,10 @@ __device__ __forceinline__ uint32_t pick_row_half(const uint32_t (&rm)[4], int k
   return ((k & 4) ? hi : lo) & 0xFFFFu;
 }
 
+__device__ __forceinline__ int32_t tile_row(const QuantParams& p, int32_t t) {
+  return p.tiles_c == 1 ? t : (int32_t)(__umulhi((uint32_t)t, p.tc_magic) >> p.tc_shift);
+}
+
 // Byte offset, inside one 512-byte chunk of a blocked scale array, of the
 // chunk's row r (0..127).
 __device__ __forceinline__ uint32_t blocked_in_chunk(int r) {
@@ -261,10 +275,10 @@ __device__ __forceinline__ void qt_readout(const QuantParams& p, const uint8_t* 
 // RSHFL selects how the row scales reach the threads (ROW without BLOCK):
 // the 16 lanes of a row group reduce-scatter the row maxima, one lane per row
 // derives the exponent and the others read 2^-e with shuffles (fewer
-// instructions: faster when each CTA has only a few tiles), or every lane
-// gets every row's amax by a butterfly and derives the exponents of its 8
-// rows itself, two rows per word (no cross-lane latency on the encode path:
-// faster on long tile streams).  Both give identical results.
+// instructions; the form every activation launch uses), or every lane gets
+// every row's amax by a butterfly and derives the exponents of its 8 rows
+// itself, two rows per word (no cross-lane latency on the encode path; it was
+// faster on long streams at two CTAs per SM).  Both give identical results.
 //
 // Addressing is kept out of the per-element work: every output pointer is
 // formed once per tile from per-thread constants and advanced by its stride,
@@ -308,7 +322,7 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
     for (int32_t k = 0; k < STAGES; ++k) {
       const int32_t t = (int32_t)blockIdx.x + k * (int32_t)gridDim.x;
       if (t >= p.tiles) break;
-      const int32_t r = t / p.tiles_c;
+      const int32_t r = tile_row(p, t);
       tma_prefetch_l2_2d(&tm_x, (t - r * p.tiles_c) * 128, r * 128);
     }
   }
@@ -330,7 +344,7 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
     if (by_ticket && ticket == (uint32_t)(p.tiles - 1)) atomicExch(p.ctr, 0u);
     ++p_it;
     if (t < p.tiles) {
-      const int32_t r = t / p.tiles_c, c = t - r * p.tiles_c;
+      const int32_t r = tile_row(p, t), c = t - r * p.tiles_c;
       tile_rc[s] = make_int2(r, c);
       mbar_arrive_expect_tx(&full[s], kQTileBytes);
       tma_load_2d<1>(tiles + s * kQTileBytes, &tm_x, c * 128, r * 128, smem_u32(&full[s]));

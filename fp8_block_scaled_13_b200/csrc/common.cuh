@@ -361,6 +361,18 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* s
                : "memory");
 }
 
+// TMA tensor store of a 3-D box from shared memory (dense in the order of the
+// tensor map's dimensions, laid out by its swizzle mode) to global memory;
+// joins the thread's current bulk async-group.  Elements outside the tensor
+// are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* src, int32_t x,
+                                             int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
+               : "memory");
+}
+
 // TMA tensor reduce-add of a 2-D box from shared memory into global memory
 // (element type from the tensor map; FP32 adds are done by the memory system,
 // one add per element per call).  Joins the thread's current bulk async-group.

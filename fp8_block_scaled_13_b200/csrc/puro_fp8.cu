@@ -140,6 +140,24 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, co
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return PURO_ERR_CUDA;
+  // The transposed codes qt [cols][ld_qt] as a 3-D tensor {qt_cols, cols/8,
+  // 8} with strides {1, 8 ld_qt, ld_qt} bytes and 128-byte swizzle: a 128 x
+  // 16 x 8 box is one tile, its transposed row 8 c_hi + c_lo at staging row
+  // 16 c_lo + c_hi, which is how the kernel stages it.  qt_cols: the bytes of
+  // a transposed row that are written (rows rounded up to 16 for
+  // activations, whose padding codes are 0; n for weights).
+  CUtensorMap mqt = m;
+  if (COL) {
+    const int64_t qt_cols = BLOCK ? p.rows : (p.rows + 15) / 16 * 16;
+    cuuint64_t qdims[3] = {(cuuint64_t)qt_cols, (cuuint64_t)(p.cols / 8), 8};
+    cuuint64_t qstrides[2] = {(cuuint64_t)p.ld_qt * 8, (cuuint64_t)p.ld_qt};
+    cuuint32_t qbox[3] = {128, 16, 8};
+    cuuint32_t qestr[3] = {1, 1, 1};
+    if (g_encode(&mqt, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p.qt, qdims, qstrides, qbox, qestr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return PURO_ERR_CUDA;
+  }
   auto kern = puro::quant_kernel<ROW, COL, BLOCK, RSHFL, STAGES>;
   constexpr uint32_t smem = puro::quant_smem_bytes<STAGES>();
   // per device, once (threads racing on the first call both set the same value)
@@ -161,7 +179,7 @@ int launch_quant_cfg(const void* x, int64_t ld_x, const puro::QuantParams& p, co
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, m, p) != cudaSuccess) return PURO_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, m, mqt, p) != cudaSuccess) return PURO_ERR_CUDA;
   return launch_status();
 }
 

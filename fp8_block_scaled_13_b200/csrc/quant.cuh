@@ -22,11 +22,12 @@
 // tid%16) holds rows 8i..8i+7 and columns 8j..8j+7.  From those registers:
 //   ROW   : row amax by a 16-lane shuffle reduction; codes stored in place.
 //   COL   : column amax by a shuffle + shared-memory reduction over the 8
-//           warps; codes transposed through an XOR-swizzled 16 KB shared tile
-//           (conflict-free 8-byte writes, 16-byte reads) and written out as
-//           128-byte rows of the transposed matrix.  The transposed tile is
-//           double-buffered and copied out during the next tile, after the
-//           barrier every tile starts with anyway.
+//           warps; codes transposed through a swizzled 16 KB shared tile
+//           (conflict-free 8-byte writes) that one TMA tensor store writes
+//           out (a 3-D view of the transposed matrix whose swizzle matches
+//           the staging layout).  The transposed tile is double-buffered and
+//           stored at the start of the next tile, after the barrier every
+//           tile starts with anyway.
 //   BLOCK : one amax over the whole tile (128x128 weight block); codes written
 //           in place and, optionally, transposed.
 // Per tile the block meets at three barriers: stage consumed (which also
@@ -250,28 +251,6 @@ __device__ __forceinline__ uint32_t blocked_in_chunk(int r) {
   return static_cast<uint32_t>((r & 31) * 16 + ((r >> 5) & 3) * 4);
 }
 
-// The transposed codes of tile (r0, c0), staged in qt_s, to global memory:
-// thread (c_base, part) writes 16 rows' codes (one 16-byte unit) of four
-// transposed rows.  Row c of the staged tile holds the 8-byte chunk of rows
-// 8i..8i+7 at position i ^ 2(c/8 & 7), so 16-byte unit u of row c is at
-// position u ^ (c/8 & 7).  Units that start past the last row are skipped
-// (the units that are written cover rows up to the next multiple of 16; rows
-// past the end read zeros, whose codes are 0, the padding the layout wants).
-__device__ __forceinline__ void qt_readout(const QuantParams& p, const uint8_t* qt_s, int32_t r0,
-                                           int32_t c0, int tid) {
-  const int c_base = tid >> 3, part = tid & 7;
-  if (r0 + 16 * part >= p.rows) return;
-  uint8_t* dst = p.qt + (int64_t)(c0 + c_base) * p.ld_qt + (r0 + 16 * part);
-  const int64_t pass_stride = (int64_t)32 * p.ld_qt;
-#pragma unroll
-  for (int pass = 0; pass < 4; ++pass) {
-    const int c = pass * 32 + c_base;
-    const int unit = part ^ ((c >> 3) & 7);
-    *reinterpret_cast<uint4*>(dst) = lds_v4(qt_s + c * 128 + (unit << 4));
-    dst += pass_stride;
-  }
-}
-
 // RSHFL selects how the row scales reach the threads (ROW without BLOCK):
 // the 16 lanes of a row group reduce-scatter the row maxima, one lane per row
 // derives the exponent and the others read 2^-e with shuffles (fewer
@@ -285,7 +264,8 @@ __device__ __forceinline__ void qt_readout(const QuantParams& p, const uint8_t* 
 // and the ragged-edge tests are one 32-bit compare against a per-tile count.
 template <bool ROW, bool COL, bool BLOCK, bool RSHFL, int STAGES>
 __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
-    quant_kernel(const __grid_constant__ CUtensorMap tm_x, const QuantParams p) {
+    quant_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_qt,
+                 const QuantParams p) {
   constexpr int kWarps = kQThreads / 32;
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -312,6 +292,7 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_x);
+    if (COL) prefetch_tmap(&tm_qt);
   }
   __syncthreads();
   if (tid == 0) {
@@ -382,7 +363,15 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
     // read the same end marker)
     if (__syncthreads_or(!ok) || tr < 0) break;
     if (tid == 0) issue_next();
-    if (COL && it > 0) qt_readout(p, qt_buf + ((it - 1) & 1) * kQtTileBytes, prev_r0, prev_c0, tid);
+    if (COL && it > 0 && tid == 0) {
+      // the previous tile's transposed codes (their writers fenced them for
+      // the async proxy before the barrier above) out by one tensor store;
+      // then make sure the store before it has finished reading the buffer
+      // this tile's codes go to
+      tma_store_3d(&tm_qt, qt_buf + ((it - 1) & 1) * kQtTileBytes, prev_r0, prev_c0 >> 3, 0);
+      bulk_commit_group();
+      bulk_wait_group_read<1>();
+    }
 
     // ---- magnitudes: per-row amax of this thread's 8 columns (two rows per
     // word) and per-column-pair amax of its 8 rows
@@ -544,19 +533,24 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
         cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
       }
       uint8_t* qt_s = qt_buf + (it & 1) * kQtTileBytes;
-      // row (8j+l) of the transposed tile: this thread's 8 codes go to 8-byte
-      // chunk i ^ 2(j & 7), so that a 16-byte unit holds two consecutive
-      // chunks in order while the 32 stores of a warp fill 16 distinct chunk
-      // positions twice (two wavefronts, the minimum for 256 bytes)
-      uint8_t* dst = qt_s + (8 * j) * 128 + ((i ^ (2 * (j & 7))) << 3);
-      *reinterpret_cast<uint2*>(dst + 0 * 128) = encode_col8<0>(v, bf16_bits(cs[0]));
-      *reinterpret_cast<uint2*>(dst + 1 * 128) = encode_col8<1>(v, bf16_bits(cs[1]));
-      *reinterpret_cast<uint2*>(dst + 2 * 128) = encode_col8<2>(v, bf16_bits(cs[2]));
-      *reinterpret_cast<uint2*>(dst + 3 * 128) = encode_col8<3>(v, bf16_bits(cs[3]));
-      *reinterpret_cast<uint2*>(dst + 4 * 128) = encode_col8<4>(v, bf16_bits(cs[4]));
-      *reinterpret_cast<uint2*>(dst + 5 * 128) = encode_col8<5>(v, bf16_bits(cs[5]));
-      *reinterpret_cast<uint2*>(dst + 6 * 128) = encode_col8<6>(v, bf16_bits(cs[6]));
-      *reinterpret_cast<uint2*>(dst + 7 * 128) = encode_col8<7>(v, bf16_bits(cs[7]));
+      // Transposed row c = 8j + l of the tile sits at staging row 16l + j,
+      // and this thread's 8 codes of it (rows 8i..8i+7) in 8-byte chunk
+      // i ^ 2(j & 7), i.e. 16-byte unit (i/2) ^ (j & 7): the 32 stores of a
+      // warp fill 16 distinct chunk positions twice (two wavefronts, the
+      // minimum for 256 bytes).  This is the layout the tensor store reads:
+      // its map views the transposed codes as {rows, cols/8 (stride 8 rows),
+      // 8 (stride 1 row)}, so staging row 16l + j is transposed row 8j + l,
+      // and its 128-byte swizzle XORs unit u with staging row & 7 = j & 7.
+      uint8_t* dst = qt_s + j * 128 + ((i ^ (2 * (j & 7))) << 3);
+      *reinterpret_cast<uint2*>(dst + 0 * 2048) = encode_col8<0>(v, bf16_bits(cs[0]));
+      *reinterpret_cast<uint2*>(dst + 1 * 2048) = encode_col8<1>(v, bf16_bits(cs[1]));
+      *reinterpret_cast<uint2*>(dst + 2 * 2048) = encode_col8<2>(v, bf16_bits(cs[2]));
+      *reinterpret_cast<uint2*>(dst + 3 * 2048) = encode_col8<3>(v, bf16_bits(cs[3]));
+      *reinterpret_cast<uint2*>(dst + 4 * 2048) = encode_col8<4>(v, bf16_bits(cs[4]));
+      *reinterpret_cast<uint2*>(dst + 5 * 2048) = encode_col8<5>(v, bf16_bits(cs[5]));
+      *reinterpret_cast<uint2*>(dst + 6 * 2048) = encode_col8<6>(v, bf16_bits(cs[6]));
+      *reinterpret_cast<uint2*>(dst + 7 * 2048) = encode_col8<7>(v, bf16_bits(cs[7]));
+      fence_proxy_async_smem();  // visible to the tensor store after the next barrier
       prev_r0 = r0;
       prev_c0 = c0;
     }
@@ -572,11 +566,15 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
     // of the next iteration, which no thread passes before every thread has
     // finished this tile.
   }
-  // the last tile's transposed codes (if every wait succeeded)
+  // the last tile's transposed codes (if every wait succeeded), and every
+  // tensor store complete before the block exits
   if (COL && it > 0) {
-    if (!__syncthreads_or(*abort_flag != 0))
-      qt_readout(p, qt_buf + ((it - 1) & 1) * kQtTileBytes, prev_r0, prev_c0, tid);
+    if (!__syncthreads_or(*abort_flag != 0) && tid == 0) {
+      tma_store_3d(&tm_qt, qt_buf + ((it - 1) & 1) * kQtTileBytes, prev_r0, prev_c0 >> 3, 0);
+      bulk_commit_group();
+    }
   }
+  if (COL && tid == 0) bulk_wait_group<0>();
   // Copies are only issued for tiles this CTA processes, and each one was
   // waited for above, unless a wait gave up; then let the outstanding ones
   // land (bounded) before the block exits.

@@ -73,14 +73,14 @@ LOADED_WATTS = 500.0         # board power above which a clock sample counts as 
 # kernel changes, until it is captured again.
 TRAFFIC_WORKLOAD = "full_block_m32768"
 TRAFFIC_BYTES = {
-    "qkv.quant_weight": 12_600_000, "qkv.quant_x": 210_600_000, "qkv.fprop": 222_300_000,
-    "qkv.quant_dy": 346_100_000, "qkv.dgrad_wgrad": 498_100_000,
-    "o_proj.quant_weight": 8_400_000, "o_proj.quant_x": 210_700_000, "o_proj.fprop": 156_600_000,
-    "o_proj.quant_dy": 210_400_000, "o_proj.dgrad_wgrad": 326_000_000,
-    "gate_up.quant_weight": 50_900_000, "gate_up.quant_x": 211_500_000, "gate_up.fprop": 876_200_000,
-    "gate_up.quant_dy": 1_560_600_000, "gate_up.dgrad_wgrad": 2_231_100_000,
-    "down.quant_weight": 25_200_000, "down.quant_x": 751_200_000, "down.fprop": 325_400_000,
-    "down.quant_dy": 210_600_000, "down.dgrad_wgrad": 1_001_800_000,
+    "qkv.quant_weight": 12_600_000, "qkv.quant_x": 209_600_000, "qkv.fprop": 221_700_000,
+    "qkv.quant_dy": 345_000_000, "qkv.dgrad_wgrad": 497_300_000,
+    "o_proj.quant_weight": 8_400_000, "o_proj.quant_x": 213_000_000, "o_proj.fprop": 156_300_000,
+    "o_proj.quant_dy": 209_400_000, "o_proj.dgrad_wgrad": 328_300_000,
+    "gate_up.quant_weight": 50_900_000, "gate_up.quant_x": 209_900_000, "gate_up.fprop": 883_800_000,
+    "gate_up.quant_dy": 1_559_100_000, "gate_up.dgrad_wgrad": 1_762_200_000,
+    "down.quant_weight": 25_200_000, "down.quant_x": 750_900_000, "down.fprop": 325_300_000,
+    "down.quant_dy": 209_200_000, "down.dgrad_wgrad": 994_600_000,
 }
 
 

@@ -209,9 +209,12 @@ int launch_quant(const void* x, int64_t ld_x, const puro::QuantParams& p, const 
     ps.tc_magic = (uint32_t)(((uint64_t(1) << (31 + l)) + (uint64_t)ps.tiles_c - 1) / (uint64_t)ps.tiles_c);
     ps.tc_shift = l - 1;
   }
-  if (BLOCK) return launch_quant_cfg<ROW, COL, BLOCK, false, 2>(x, ld_x, ps, dev, stream);
-  if (short_stream) return launch_quant_cfg<ROW, COL, BLOCK, ROW, 2>(x, ld_x, ps, dev, stream);
-  return launch_quant_cfg<ROW, COL, BLOCK, ROW, 1>(x, ld_x, ps, dev, stream);
+  if constexpr (BLOCK) {
+    return launch_quant_cfg<ROW, COL, BLOCK, false, 2>(x, ld_x, ps, dev, stream);
+  } else {
+    if (short_stream) return launch_quant_cfg<ROW, COL, BLOCK, ROW, 2>(x, ld_x, ps, dev, stream);
+    return launch_quant_cfg<ROW, COL, BLOCK, ROW, 1>(x, ld_x, ps, dev, stream);
+  }
 }
 
 // ------------------------------------------------------------------ gemm

@@ -231,16 +231,6 @@ __device__ __forceinline__ uint4 lds_v4(const uint8_t* p) {
   return *reinterpret_cast<const uint4*>(p);
 }
 
-// Row k's amax (BF16 bits) out of the four row-pair words of row_amax, for a
-// lane-dependent k: byte permutes pick the half-word (a plain or selected
-// array index would be lowered to a local-memory round trip).
-__device__ __forceinline__ uint32_t pick_row_half(const uint32_t (&rm)[4], int k) {
-  const uint32_t b = 2u * static_cast<uint32_t>(k & 3);  // byte of the half within a word pair
-  const uint32_t sel = b | ((b + 1u) << 4);
-  const uint32_t lo = __byte_perm(rm[0], rm[1], sel), hi = __byte_perm(rm[2], rm[3], sel);
-  return ((k & 4) ? hi : lo) & 0xFFFFu;
-}
-
 __device__ __forceinline__ int32_t tile_row(const QuantParams& p, int32_t t) {
   return p.tiles_c == 1 ? t : (int32_t)(__umulhi((uint32_t)t, p.tc_magic) >> p.tc_shift);
 }
@@ -251,13 +241,12 @@ __device__ __forceinline__ uint32_t blocked_in_chunk(int r) {
   return static_cast<uint32_t>((r & 31) * 16 + ((r >> 5) & 3) * 4);
 }
 
-// RSHFL selects how the row scales reach the threads (ROW without BLOCK):
+// RSHFL marks the row-scale form of activation launches (ROW without BLOCK):
 // the 16 lanes of a row group reduce-scatter the row maxima, one lane per row
-// derives the exponent and the others read 2^-e with shuffles (fewer
-// instructions; the form every activation launch uses), or every lane gets
-// every row's amax by a butterfly and derives the exponents of its 8 rows
-// itself, two rows per word (no cross-lane latency on the encode path; it was
-// faster on long streams at two CTAs per SM).  Both give identical results.
+// derives the exponent and the others read 2^-e with shuffles.  (An earlier
+// form had every lane derive its own 8 rows' exponents after a butterfly:
+// faster at two CTAs per SM on long streams, 7% more instructions, and slower
+// at three CTAs per SM.)  Weight blocks take one scale for the whole tile.
 //
 // Addressing is kept out of the per-element work: every output pointer is
 // formed once per tile from per-thread constants and advanced by its stride,
@@ -266,6 +255,7 @@ template <bool ROW, bool COL, bool BLOCK, bool RSHFL, int STAGES>
 __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
     quant_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_qt,
                  const QuantParams p) {
+  static_assert(!ROW || BLOCK || RSHFL, "activation row scales are shared by shuffles");
   constexpr int kWarps = kQThreads / 32;
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -340,7 +330,6 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
     for (int k = 0; k < STAGES; ++k) issue_next();
 
   // per-thread constants of the output addressing
-  const uint32_t s_own_row = blocked_in_chunk(8 * i + (j & 7));    // row scale byte (j < 8)
   const uint32_t s_half_chunk = blocked_in_chunk(8 * i + (j >> 1));  // the same, row j >> 1
   const uint32_t st_in_chunk = blocked_in_chunk(2 * (tid & 63));     // column scale bytes (tid < 64)
 
@@ -486,32 +475,11 @@ __global__ void __launch_bounds__(kQThreads, STAGES == 1 ? 3 : 2)
           qrow += p.ld_q;
         }
       } else {
-        // every lane gets every row's amax (butterfly) and derives its 8 rows'
-        // exponents two at a time; lane j < 8 stores row 8i + j's scale byte
-        float sc[8];
-        if (BLOCK) {
-          const float f = __uint_as_float(static_cast<uint32_t>(127 - e_blk) << 23);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) sc[k] = f;
-        } else {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-#pragma unroll
-            for (int off = 8; off >= 1; off >>= 1)
-              rowmax[q] = __vmaxu2(rowmax[q], __shfl_xor_sync(0xFFFFFFFFu, rowmax[q], off));
-            const uint32_t k2 = scale_k2(rowmax[q]);
-            sc[2 * q] = scale_lo(k2);
-            sc[2 * q + 1] = scale_hi(k2);
-          }
-          if (j < 8) {
-            const uint32_t a = pick_row_half(rowmax, j);
-            const uint32_t b = scale_bytes2(a, scale_k2(a)) & 0xFFu;
-            p.s[((int64_t)tr * p.s_g4 + (tc >> 2)) * 512 + (tc & 3) + s_own_row] = static_cast<uint8_t>(b);
-          }
-        }
+        // a weight block: one scale for every row
+        const uint16_t sb = bf16_bits(__uint_as_float(static_cast<uint32_t>(127 - e_blk) << 23));
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint2 o = encode_row8(v[k], bf16_bits(sc[k]));
+          const uint2 o = encode_row8(v[k], sb);
           if (k < nrow) *reinterpret_cast<uint2*>(qrow) = o;
           qrow += p.ld_q;
         }

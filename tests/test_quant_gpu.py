@@ -260,3 +260,21 @@ def test_tile_counter_graph_replays(fp8):
         assert not xq.work.any(), "tile counter not reset"
         assert _same(ref, _outs(xq))
     del g
+
+
+@pytest.mark.parametrize("case", ["static_edge", "ticket_edge", "ticket_narrow3_ragged"])
+def test_tile_counter_threshold(fp8, oracle_mod, case):
+    """Both sides of the ticket threshold (16 tiles per SM), against the oracle
+    over the whole tensor: the last static-schedule size, the first ticket
+    size (one tile per row of tiles, so the tile decode is the identity), and
+    a three-tile-wide ragged input just past the threshold (multiply-shift
+    decode)."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    limit = 16 * sms
+    rows, cols = {"static_edge": (limit * 128, 128),
+                  "ticket_edge": ((limit + 1) * 128, 128),
+                  "ticket_narrow3_ragged": ((limit // 3 + 1) * 128 - 37, 384)}[case]
+    tiles = -(-rows // 128) * (cols // 128)
+    assert (tiles > limit) == (case != "static_edge")
+    xq = _check_all(fp8, oracle_mod, _rand((rows, cols), tiles), "both")
+    assert not xq.work.any(), "tile counter not reset"

@@ -25,6 +25,7 @@ def _round16(n: int) -> int:
     return (n + 15) // 16 * 16
 
 
+@functools.lru_cache(maxsize=1024)
 def blocked_scale_bytes(rows: int, groups: int) -> int:
     return _lib.puro_fp8_blocked_scale_bytes(rows, groups)
 
@@ -33,18 +34,29 @@ def _blocked(rows: int, groups: int, dev) -> torch.Tensor:
     return torch.empty(max(blocked_scale_bytes(rows, groups), 16), dtype=torch.uint8, device=dev)
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream() -> int:
+    """The current CUDA stream of the current device, as a cudaStream_t value."""
+    if _raw_stream is not None:
+        return _raw_stream(torch.cuda.current_device())
     return torch.cuda.current_stream().cuda_stream
 
 
+_FIELD_NAMES: dict = {}
+
+
 def _tensors(obj):
+    """The tensors of a wrapper argument: a tensor, or a dataclass's tensor fields."""
     if isinstance(obj, torch.Tensor):
-        yield obj
-    elif dataclasses.is_dataclass(obj) and not isinstance(obj, type):
-        for f in dataclasses.fields(obj):
-            v = getattr(obj, f.name)
-            if isinstance(v, torch.Tensor):
-                yield v
+        return (obj,)
+    names = _FIELD_NAMES.get(type(obj))
+    if names is None:
+        if not dataclasses.is_dataclass(obj) or isinstance(obj, type):
+            return ()
+        names = _FIELD_NAMES[type(obj)] = tuple(f.name for f in dataclasses.fields(obj))
+    return tuple(v for v in (getattr(obj, n) for n in names) if isinstance(v, torch.Tensor))
 
 
 def _on_operand_device(fn):
@@ -54,11 +66,16 @@ def _on_operand_device(fn):
     several devices are refused."""
     @functools.wraps(fn)
     def wrapper(*args, **kwargs):
-        devs = {t.device for a in (*args, *kwargs.values()) for t in _tensors(a)}
-        if len(devs) > 1:
-            raise ValueError("%s: operands are on different devices (%s)"
-                             % (fn.__name__, ", ".join(sorted(str(d) for d in devs))))
-        dev = devs.pop() if devs else None
+        operands = (*args, *kwargs.values()) if kwargs else args
+        dev = None
+        for a in operands:
+            for t in _tensors(a):
+                if dev is None:
+                    dev = t.device
+                elif t.device != dev:
+                    devs = {t.device for a in operands for t in _tensors(a)}
+                    raise ValueError("%s: operands are on different devices (%s)"
+                                     % (fn.__name__, ", ".join(sorted(str(d) for d in devs))))
         if dev is not None and dev.type == "cuda" and dev.index != torch.cuda.current_device():
             with torch.cuda.device(dev):
                 return fn(*args, **kwargs)
@@ -165,12 +182,17 @@ class QuantWeight:
     s_bwd: torch.Tensor | None = None  # blocked: k rows x n/128 groups (dgrad B scales)
 
 
+_LAYOUTS = {"rowwise": _lib.PURO_ROWWISE, "colwise": _lib.PURO_COLWISE, "both": _lib.PURO_BOTH}
+
+
 @_on_operand_device
 def quant_act(x: torch.Tensor, layout: str = "both", out: QuantAct | None = None) -> QuantAct:
     """1x128 quantization of an activation/gradient x [rows, cols] (BF16)."""
     _require(x, torch.bfloat16, "x")
     rows, cols = x.shape
-    flag = {"rowwise": _lib.PURO_ROWWISE, "colwise": _lib.PURO_COLWISE, "both": _lib.PURO_BOTH}[layout]
+    flag = _LAYOUTS.get(layout)
+    if flag is None:
+        raise ValueError("layout must be one of %s, got %r" % (", ".join(_LAYOUTS), layout))
     dev = x.device
     if out is None:
         out = QuantAct(rows, cols)

@@ -213,6 +213,8 @@ def test_wrapper_rejects_missing_layouts_and_bad_buffers(fp8):
         fp8.quant_act(x[:128].contiguous(), "rowwise", out=x_row)   # made for another shape
     with pytest.raises(ValueError):
         fp8.quant_weight(w[:128].contiguous(), out=wq)
+    with pytest.raises(ValueError, match="layout"):
+        fp8.quant_act(x, "row")                                 # unknown layout name
     # reusing a matching result works and gives the same codes
     again = fp8.quant_act(x, "rowwise", out=fp8.QuantAct(256, 384, torch.empty_like(x_row.q),
                                                           torch.empty_like(x_row.s)))

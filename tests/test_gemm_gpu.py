@@ -251,3 +251,23 @@ def test_wrapper_rejects_short_scale_buffers(fp8):
     with pytest.raises(ValueError):
         fp8.gemm_fprop(dataclasses.replace(xq, q=xq.q[:, :256]), wq)    # codes narrower than K
     assert fp8.device_status() == 0
+
+
+def test_wrappers_launch_on_the_current_stream(fp8):
+    """The wrappers hand the library the caller's current stream: the default
+    stream, or the one a `torch.cuda.stream` context makes current.  A layer
+    run on a side stream equals the same layer on the default stream."""
+    from fp8_block_scaled_13_b200 import linear
+    assert linear._stream() == torch.cuda.current_stream().cuda_stream
+    x, w, dy = _layer(300, 256, 384, 31)
+    want = _run(fp8, x, w, dy)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        assert linear._stream() == s.cuda_stream
+        dev = torch.device("cuda")
+        xd, wd, dyd = x.to(dev), w.to(dev), dy.to(dev)
+        y, xq, wq = fp8.linear_forward(xd, wd)
+        dx, dw = fp8.linear_backward(dyd, xq, wq)
+    s.synchronize()
+    for a, b in zip((y, dx, dw), want):
+        assert torch.equal(a, b)

@@ -207,12 +207,16 @@ def _long_stream(rows, cols):
 
 
 @pytest.mark.parametrize("rows,cols,layout", [(40000, 1024, "both"), (33001, 2048, "rowwise"),
-                                              (20000, 2048, "colwise")])
+                                              (20000, 2048, "colwise"),
+                                              (300, 128 * 3001, "both"),   # 3001 column tiles
+                                              (1000003, 128, "both")])     # one column tile
 def test_tile_counter_long_streams(fp8, oracle_mod, rows, cols, layout):
     """Long inputs (more than 16 tiles per SM) hand their tiles out by ticket
     from the output's counter: the oracle's bytes over the whole tensor (ragged
     last row tile included), the same bytes as the static schedule, and the
-    counter back at zero after every call."""
+    counter back at zero after every call.  The last two shapes take the tile
+    decode (row tile = ticket tile / column tiles, by multiply-shift) to an odd
+    divisor of 3001 and to the single-column-tile case."""
     assert _long_stream(rows, cols)
     x = _rand((rows, cols), rows + cols)
     xq = _check_all(fp8, oracle_mod, x, layout)
